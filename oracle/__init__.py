@@ -1,0 +1,124 @@
+"""ctypes front-end of the CPU oracle (oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
+benchmark's CPU-baseline leg; never by the library's product path.  It shares
+no code with the CUDA path.  Inputs are numpy arrays in the library's boundary
+layouts (see oracle.c for the definition and the citations).
+"""
+from __future__ import annotations
+
+import contextlib
+import ctypes as C
+import os
+
+import numpy as np
+
+from .build import build
+
+_lib = None
+
+
+def load(path: str):
+    """Load one compiled copy of oracle.c and declare its signatures."""
+    L = C.CDLL(path)
+    P = C.c_void_p
+    i = C.c_int
+    L.fp8o_e4m3_value.restype = C.c_double
+    L.fp8o_e4m3_value.argtypes = [C.c_uint8]
+    L.fp8o_bf16_rne.restype = C.c_uint16
+    L.fp8o_bf16_rne.argtypes = [C.c_double]
+    L.fp8o_gemm_nt.restype = i
+    L.fp8o_gemm_nt.argtypes = [P, P, i, P, P, i, i, i, P, i, P, P, i]
+    L.fp8o_m_grouped_contiguous.restype = i
+    L.fp8o_m_grouped_contiguous.argtypes = [P, P, i, P, P, P, i, i, i, i, P, i, P, P, i]
+    L.fp8o_m_grouped_masked.restype = i
+    L.fp8o_m_grouped_masked.argtypes = [P, P, i, P, P, P, i, i, i, i, P, P, i]
+    return L
+
+
+@contextlib.contextmanager
+def using(path: str):
+    """Temporarily route every call to another build of oracle.c (used by the
+    mutation tests, which plant mistakes in a copy of the source)."""
+    global _lib
+    saved = lib()
+    _lib = load(path)
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = load(build())
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+def e4m3_value(code: int) -> float:
+    return lib().fp8o_e4m3_value(int(code))
+
+
+def bf16_rne(x: float) -> int:
+    return lib().fp8o_bf16_rne(float(x))
+
+
+def gemm_nt(A, sa, ld_sa, B, sb, M, N, K, rows=None, nthreads=None, out_exact=None, out_bf16=None):
+    """Dense NT GEMM.  Returns (exact float64 [nrows, N], bf16 bits uint16 [nrows, N])."""
+    A, sa, B, sb = _c(A, np.uint8), _c(sa, np.float32), _c(B, np.uint8), _c(sb, np.float32)
+    r = None if rows is None else _c(rows, np.int32)
+    nrows = M if r is None else len(r)
+    ex = np.zeros((nrows, N), np.float64) if out_exact is None else out_exact
+    bf = np.zeros((nrows, N), np.uint16) if out_bf16 is None else out_bf16
+    rc = lib().fp8o_gemm_nt(_p(A), _p(sa), int(ld_sa), _p(B), _p(sb), int(M), int(N), int(K),
+                            _p(r), int(nrows), _p(ex), _p(bf), int(nthreads or default_threads()))
+    if rc:
+        raise ValueError("oracle: bad arguments")
+    return ex, bf
+
+
+def m_grouped_contiguous(A, sa, ld_sa, B, sb, m_indices, M, N, K, G, rows=None, nthreads=None,
+                         out_exact=None, out_bf16=None):
+    """Contiguous grouped GEMM.  Output slots of rows in skipped (-1) blocks keep
+    the values passed in (out_exact/out_bf16), default 0."""
+    A, sa, B, sb = _c(A, np.uint8), _c(sa, np.float32), _c(B, np.uint8), _c(sb, np.float32)
+    mi = _c(m_indices, np.int32)
+    r = None if rows is None else _c(rows, np.int32)
+    nrows = M if r is None else len(r)
+    ex = np.zeros((nrows, N), np.float64) if out_exact is None else out_exact
+    bf = np.zeros((nrows, N), np.uint16) if out_bf16 is None else out_bf16
+    rc = lib().fp8o_m_grouped_contiguous(_p(A), _p(sa), int(ld_sa), _p(B), _p(sb), _p(mi),
+                                         int(M), int(N), int(K), int(G), _p(r), int(nrows),
+                                         _p(ex), _p(bf), int(nthreads or default_threads()))
+    if rc:
+        raise ValueError("oracle: bad arguments")
+    return ex, bf
+
+
+def m_grouped_masked(A, sa, ld_sa, B, sb, masked_m, G, Mmax, N, K, nthreads=None,
+                     out_exact=None, out_bf16=None):
+    """Masked grouped GEMM over [G, Mmax, N].  Rows m >= masked_m[g] keep the
+    values passed in (default 0)."""
+    A, sa, B, sb = _c(A, np.uint8), _c(sa, np.float32), _c(B, np.uint8), _c(sb, np.float32)
+    mm = _c(masked_m, np.int32)
+    ex = np.zeros((G, Mmax, N), np.float64) if out_exact is None else out_exact
+    bf = np.zeros((G, Mmax, N), np.uint16) if out_bf16 is None else out_bf16
+    rc = lib().fp8o_m_grouped_masked(_p(A), _p(sa), int(ld_sa), _p(B), _p(sb), _p(mm), int(G),
+                                     int(Mmax), int(N), int(K), _p(ex), _p(bf),
+                                     int(nthreads or default_threads()))
+    if rc:
+        raise ValueError("oracle: bad arguments")
+    return ex, bf

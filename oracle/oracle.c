@@ -1,0 +1,299 @@
+/*
+ * oracle.c -- plain CPU reference of the fine-grained-scaled FP8 GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the library's product path links,
+ * loads or calls this file; only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark do.  It shares no code, header, table or
+ * helper with the CUDA path.
+ *
+ * What it computes (the definition; every function below cites the passage
+ * it follows):
+ *
+ *   D[m,n] = bf16_rne( sum_{kb=0}^{KB-1}
+ *                        ( sum_{k=128kb}^{128kb+127} dec(A[m,k]) * dec(B[n,k]) )
+ *                        * sa[m,kb] * sb[n/128, kb] )
+ *
+ * A carries one FP32 scale per 1x128 row group, B one per 128x128 block
+ * (the "fine-grained scaling" of DeepSeek-V3 that DeepGEMM supports: GeekNews
+ * "DeepSeek, DeepGEMM 오픈소스 공개", topic body, first bullet), and each
+ * 128-wide K-block partial is promoted to higher precision before it is
+ * scaled and accumulated (same page, fifth bullet: CUDA-core promotion of
+ * the imprecise FP8 tensor-core accumulation).  Here the promotion target is
+ * FP64:
+ *   - a K-block partial is a sum of 128 products of e4m3 values; each product
+ *     has at most 8 significant bits and lies in [2^-18, 448^2], so the
+ *     128-term sum is exact in double;
+ *   - the partial is multiplied by (double)sa then (double)sb and added to a
+ *     double running sum, in K-block order (no reassociation);
+ *   - the result is returned unrounded (for tolerance checks) and rounded
+ *     once to bf16, round-to-nearest-even (the "bf16" of the API name,
+ *     flashmla.net "Quick Start Guide": m_grouped_gemm_fp8_fp8_bf16_nt_...).
+ *
+ * Layouts (the library's boundary layouts):
+ *   A  [M,K] e4m3 codes, K contiguous          (NT: B is [N,K], K contiguous)
+ *   sa [KB][ld_sa] float, sa[kb*ld_sa + m]     (masked: [G][KB][ld_sa])
+ *   sb [NB][KB]   float, sb[nb*KB + kb]        (grouped: [G][NB][KB])
+ *   D  [M,N]                                   (masked: [G][Mmax][N])
+ * Grouped layouts (GeekNews page, "MoE 모델을 위한 그룹화 GEMM 성능"):
+ *   contiguous: rows grouped along M with N, K shared; m_indices[r] gives the
+ *     expert of 128-row block r, -1 = no expert (rows left unwritten);
+ *   masked: only rows m < masked_m[g] of group g are computed; the rest are
+ *     left unwritten.
+ *
+ * Compiled with -ffp-contract=off so that no multiply-add is fused and every
+ * operation rounds exactly as written.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------------------
+ * e4m3 decode -- OCP 8-bit floating point, E4M3 ("fn") encoding: sign bit,
+ * 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds the
+ * subnormals m * 2^-9; S.1111.111 is NaN; there are no infinities; the
+ * largest finite value is S.1111.110 = 448.  The pages name the format
+ * (flashmla.net, "FP8 Precision Meets Industrial Rigor": fp8_e4m3/fp8_e5m2).
+ * ------------------------------------------------------------------------- */
+double fp8o_e4m3_value(uint8_t code)
+{
+    int s = code >> 7;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);               /* (m/8) * 2^(1-7) */
+    else
+        v = ldexp(8.0 + (double)m, e - 7 - 3);  /* (1 + m/8) * 2^(e-7) */
+    return s ? -v : v;
+}
+
+/* ---------------------------------------------------------------------------
+ * bf16 round-to-nearest-even of a double, one rounding.  bf16 = sign, 8-bit
+ * exponent (bias 127), 7 stored mantissa bits; subnormal quantum 2^-133.
+ * Returns the 16-bit pattern.
+ * ------------------------------------------------------------------------- */
+uint16_t fp8o_bf16_rne(double x)
+{
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    int E, e;
+    double q, n;
+    if (isnan(x))
+        return 0x7FC0;
+    if (isinf(x))
+        return sign | 0x7F80;
+    if (a == 0.0)
+        return sign;
+    (void)frexp(a, &E);          /* a = f * 2^E, f in [0.5, 1) */
+    e = E - 1;                   /* a in [2^e, 2^(e+1)) */
+    if (e < -126)
+        e = -126;                /* subnormal range shares the quantum 2^-133 */
+    q = ldexp(1.0, e - 7);
+    n = nearbyint(a / q);        /* a/q is exact (power-of-two scaling); ties to even */
+    if (n >= 256.0) {            /* mantissa carried into the exponent */
+        n = 128.0;
+        e += 1;
+    }
+    if (n < 128.0)               /* subnormal (only when e == -126) */
+        return sign | (uint16_t)n;
+    if (e + 127 >= 255)
+        return sign | 0x7F80;    /* overflow rounds to infinity */
+    return sign | (uint16_t)(((e + 127) << 7) | ((int)n - 128));
+}
+
+/* ---------------------------------------------------------------------------
+ * One output row of the definition above.  a_row: K codes of A's row;
+ * sa_col: the row's K-block scales, stride sa_stride floats apart;
+ * B: [N,K] codes; sb: [NB][KB].  Writes N doubles and N bf16 patterns.
+ * ------------------------------------------------------------------------- */
+static void row_nt(const uint8_t *a_row, const float *sa_col, long sa_stride,
+                   const uint8_t *B, const float *sb, int N, int K,
+                   double *out_exact, uint16_t *out_bf16)
+{
+    int KB = K / 128;
+    double adec[128];
+    double *acc = (double *)calloc((size_t)N, sizeof(double));
+    for (int kb = 0; kb < KB; ++kb) {
+        double s_a = (double)sa_col[(long)kb * sa_stride];
+        for (int j = 0; j < 128; ++j)
+            adec[j] = fp8o_e4m3_value(a_row[kb * 128 + j]);
+        for (int n = 0; n < N; ++n) {
+            const uint8_t *b = B + (long)n * K + (long)kb * 128;
+            double partial = 0.0;                      /* exact: see header */
+            for (int j = 0; j < 128; ++j)
+                partial += adec[j] * fp8o_e4m3_value(b[j]);
+            double s_b = (double)sb[(long)(n / 128) * KB + kb];
+            acc[n] += (partial * s_a) * s_b;
+        }
+    }
+    for (int n = 0; n < N; ++n) {
+        if (out_exact)
+            out_exact[n] = acc[n];
+        if (out_bf16)
+            out_bf16[n] = fp8o_bf16_rne(acc[n]);
+    }
+    free(acc);
+}
+
+/* ---------------------------------------------------------------------------
+ * A job = a list of output rows; each resolved to (A row, sa column, B, sb,
+ * output slot).  Threads take rows round-robin.  Rows are independent, so
+ * splitting them across threads changes no arithmetic.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    const uint8_t *a_row;
+    const float *sa_col;
+    long sa_stride;
+    const uint8_t *B;
+    const float *sb;
+    double *out_exact;
+    uint16_t *out_bf16;
+} row_task;
+
+typedef struct {
+    const row_task *tasks;
+    int ntasks, N, K, tid, nthreads;
+} worker_arg;
+
+static void *worker(void *p)
+{
+    worker_arg *w = (worker_arg *)p;
+    for (int i = w->tid; i < w->ntasks; i += w->nthreads) {
+        const row_task *t = &w->tasks[i];
+        row_nt(t->a_row, t->sa_col, t->sa_stride, t->B, t->sb, w->N, w->K,
+               t->out_exact, t->out_bf16);
+    }
+    return NULL;
+}
+
+static void run_tasks(const row_task *tasks, int ntasks, int N, int K, int nthreads)
+{
+    if (nthreads < 1)
+        nthreads = 1;
+    if (nthreads > 256)
+        nthreads = 256;
+    pthread_t th[256];
+    worker_arg args[256];
+    for (int t = 0; t < nthreads; ++t) {
+        args[t] = (worker_arg){tasks, ntasks, N, K, t, nthreads};
+        if (t > 0)
+            pthread_create(&th[t], NULL, worker, &args[t]);
+    }
+    worker(&args[0]);
+    for (int t = 1; t < nthreads; ++t)
+        pthread_join(th[t], NULL);
+}
+
+/* ---------------------------------------------------------------------------
+ * Dense NT GEMM (GeekNews page, "일반 GEMM 성능 (Dense 모델)").
+ * rows: the output rows to compute (NULL = all M rows, in order); output
+ * slot i of out_exact/out_bf16 ([nrows][N]) holds row rows[i].
+ * Returns 0, or -1 on a bad argument.
+ * ------------------------------------------------------------------------- */
+int fp8o_gemm_nt(const uint8_t *A, const float *sa, int ld_sa,
+                 const uint8_t *B, const float *sb,
+                 int M, int N, int K, const int *rows, int nrows,
+                 double *out_exact, uint16_t *out_bf16, int nthreads)
+{
+    if (K % 128 || M < 0 || N < 0 || ld_sa < M)
+        return -1;
+    if (!rows)
+        nrows = M;
+    row_task *tasks = (row_task *)malloc(sizeof(row_task) * (size_t)(nrows ? nrows : 1));
+    for (int i = 0; i < nrows; ++i) {
+        int m = rows ? rows[i] : i;
+        if (m < 0 || m >= M) {
+            free(tasks);
+            return -1;
+        }
+        tasks[i] = (row_task){A + (long)m * K, sa + m, ld_sa, B, sb,
+                              out_exact ? out_exact + (long)i * N : NULL,
+                              out_bf16 ? out_bf16 + (long)i * N : NULL};
+    }
+    run_tasks(tasks, nrows, N, K, nthreads);
+    free(tasks);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * M-grouped contiguous (GeekNews page, "연속된(contiguous) 레이아웃"): the
+ * experts' row segments are concatenated along M; 128-row block r uses expert
+ * m_indices[r]'s B [N,K] and sb [NB][KB]; blocks with m_indices[r] < 0 are
+ * skipped and their output rows are not written.
+ * B: [G][N][K]; sb: [G][NB][KB]; out rows are indexed like `rows`.
+ * ------------------------------------------------------------------------- */
+int fp8o_m_grouped_contiguous(const uint8_t *A, const float *sa, int ld_sa,
+                              const uint8_t *B, const float *sb, const int32_t *m_indices,
+                              int M, int N, int K, int G, const int *rows, int nrows,
+                              double *out_exact, uint16_t *out_bf16, int nthreads)
+{
+    if (K % 128 || M % 128 || N < 0 || G < 1 || ld_sa < M)
+        return -1;
+    int KB = K / 128, NB = (N + 127) / 128;
+    if (!rows)
+        nrows = M;
+    row_task *tasks = (row_task *)malloc(sizeof(row_task) * (size_t)(nrows ? nrows : 1));
+    int nt = 0;
+    for (int i = 0; i < nrows; ++i) {
+        int m = rows ? rows[i] : i;
+        if (m < 0 || m >= M) {
+            free(tasks);
+            return -1;
+        }
+        int g = m_indices[m / 128];
+        if (g < 0)
+            continue;                 /* skipped block: row not written */
+        if (g >= G) {
+            free(tasks);
+            return -1;
+        }
+        tasks[nt++] = (row_task){A + (long)m * K, sa + m, ld_sa,
+                                 B + (long)g * N * K, sb + (long)g * NB * KB,
+                                 out_exact ? out_exact + (long)i * N : NULL,
+                                 out_bf16 ? out_bf16 + (long)i * N : NULL};
+    }
+    run_tasks(tasks, nt, N, K, nthreads);
+    free(tasks);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * M-grouped masked (GeekNews page, "마스킹(masked) 레이아웃": a mask input
+ * says how many rows each expert really has, for CUDA-graph decode where the
+ * host does not know the counts): A [G][Mmax][K], sa [G][KB][ld_sa],
+ * B [G][N][K], sb [G][NB][KB], out [G][Mmax][N].  Group g computes rows
+ * m < min(masked_m[g], Mmax); other rows are not written.
+ * ------------------------------------------------------------------------- */
+int fp8o_m_grouped_masked(const uint8_t *A, const float *sa, int ld_sa,
+                          const uint8_t *B, const float *sb, const int32_t *masked_m,
+                          int G, int Mmax, int N, int K,
+                          double *out_exact, uint16_t *out_bf16, int nthreads)
+{
+    if (K % 128 || Mmax < 0 || N < 0 || G < 1 || ld_sa < Mmax)
+        return -1;
+    int KB = K / 128, NB = (N + 127) / 128;
+    long total = 0;
+    for (int g = 0; g < G; ++g) {
+        int mg = masked_m[g] < 0 ? 0 : (masked_m[g] > Mmax ? Mmax : masked_m[g]);
+        total += mg;
+    }
+    row_task *tasks = (row_task *)malloc(sizeof(row_task) * (size_t)(total ? total : 1));
+    int nt = 0;
+    for (int g = 0; g < G; ++g) {
+        int mg = masked_m[g] < 0 ? 0 : (masked_m[g] > Mmax ? Mmax : masked_m[g]);
+        for (int m = 0; m < mg; ++m) {
+            long orow = (long)g * Mmax + m;
+            tasks[nt++] = (row_task){A + orow * K, sa + (long)g * KB * ld_sa + m, ld_sa,
+                                     B + (long)g * N * K, sb + (long)g * NB * KB,
+                                     out_exact ? out_exact + orow * N : NULL,
+                                     out_bf16 ? out_bf16 + orow * N : NULL};
+        }
+    }
+    run_tasks(tasks, nt, N, K, nthreads);
+    free(tasks);
+    return 0;
+}
