@@ -1,0 +1,381 @@
+// api.cu -- host side of the C ABI declared in include/fp8gemm.h: argument
+// validation, per-device capability cache, TMA tensor-map encoding, kernel
+// variant table and selection, launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fp8gemm.h"
+#include "kernel.cuh"
+
+using namespace fp8g;
+
+namespace {
+
+// ---------------------------------------------------------------- variants
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, Params);
+
+struct Variant {
+  const char* name;
+  int kind;
+  bool swap;
+  int bnc, stages, split;
+  KernelFn fn;
+  int smem;
+};
+
+template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT>
+Variant make_variant(const char* name) {
+  return Variant{name, KIND, kSwap, BNC, STAGES, SPLIT,
+                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT>,
+                 Layout<kSwap, BNC, STAGES, SPLIT>::kSmemAlloc};
+}
+
+const Variant kVariants[] = {
+    make_variant<true, 64, 7, kDense, 8>("dense_nlanes_bn64_st7_splitk8"),
+    make_variant<true, 64, 8, kDense, 1>("dense_nlanes_bn64_st8"),
+    make_variant<true, 128, 6, kDense, 1>("dense_nlanes_bn128_st6"),
+    make_variant<false, 128, 6, kDense, 1>("dense_mlanes_bn128_st6"),
+    make_variant<true, 128, 6, kContiguous, 1>("contiguous_nlanes_bn128_st6"),
+    make_variant<false, 128, 6, kContiguous, 1>("contiguous_mlanes_bn128_st6"),
+    make_variant<true, 64, 8, kMasked, 1>("masked_nlanes_bn64_st8"),
+    make_variant<true, 128, 6, kMasked, 1>("masked_nlanes_bn128_st6"),
+    make_variant<false, 128, 6, kMasked, 1>("masked_mlanes_bn128_st6"),
+};
+constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
+enum : int {
+  V_DENSE_SPLIT = 0,
+  V_DENSE_N64 = 1,
+  V_DENSE_N128 = 2,
+  V_DENSE_M128 = 3,
+  V_CONTIG_N128 = 4,
+  V_CONTIG_M128 = 5,
+  V_MASKED_N64 = 6,
+  V_MASKED_N128 = 7,
+  V_MASKED_M128 = 8,
+};
+
+std::atomic<int> g_override{-1};
+thread_local int t_last_variant = -1;
+
+// ---------------------------------------------------------------- devices
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int sms = 0;
+  int max_smem_optin = 0;
+  bool attr_set[kNumVariants] = {};
+  int max_clusters[kNumVariants] = {};  // split variants: co-resident clusters
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8G_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return FP8G_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);
+    d.probed = true;
+  }
+  *out = &d;
+  return d.supported ? FP8G_OK : FP8G_ERR_UNSUPPORTED;
+}
+
+// Opt the variant into its shared-memory size on this device (once).
+int prepare_variant(DeviceInfo* d, int v) {
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (d->attr_set[v]) return FP8G_OK;
+  const Variant& V = kVariants[v];
+  if (V.smem > d->max_smem_optin) return FP8G_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(V.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           V.smem) != cudaSuccess)
+    return FP8G_ERR_CUDA;
+  if (V.split > 1) {
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(V.fn), cudaFuncAttributeNonPortableClusterSizeAllowed,
+                             V.split > 8 ? 1 : 0) != cudaSuccess)
+      return FP8G_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = V.split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(V.split * 64, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = V.smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(V.fn), &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    d->max_clusters[v] = n;
+  }
+  d->attr_set[v] = true;
+  return FP8G_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 3-D map (dim0 innermost).  strides are in bytes for dims 1 and 2.
+int encode3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+             uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FP8G_ERR_CUDA;
+  const cuuint64_t dims[3] = {d0, std::max<uint64_t>(d1, 1), std::max<uint64_t>(d2, 1)};
+  const cuuint64_t strides[2] = {s1, s2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8G_OK : FP8G_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- validation
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_shapes(int rows, int N, int K, int ld_sa) {
+  if (rows < 0 || N < 0 || K <= 0 || K % 128 != 0 || K > 128 * kKBMax) return FP8G_ERR_INVALID_ARG;
+  if (ld_sa < rows || ld_sa < 1) return FP8G_ERR_INVALID_ARG;
+  if (N % 8 != 0 || ld_sa % 4 != 0) return FP8G_ERR_MISALIGNED;
+  return FP8G_OK;
+}
+
+int check_ptrs(const uint8_t* A, const float* sa, const uint8_t* B, const float* sb, const uint16_t* D) {
+  if (!A || !sa || !B || !sb || !D) return FP8G_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(sa, 16) || !aligned(D, 16) || !aligned(sb, 4))
+    return FP8G_ERR_MISALIGNED;
+  return FP8G_OK;
+}
+
+struct Problem {
+  int kind;
+  const uint8_t* A;
+  const float* sa;
+  int ld_sa;
+  const uint8_t* B;
+  const float* sb;
+  uint16_t* D;
+  const int32_t* idx;  // m_indices or masked_m
+  int M;               // rows (Mmax for masked)
+  int N, K, G;
+  int expected_m;
+};
+
+int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
+  const Variant& V = kVariants[v];
+  if (V.kind != P.kind) return FP8G_ERR_UNSUPPORTED;
+  if (P.kind == kContiguous && V.swap && V.bnc != 128) return FP8G_ERR_UNSUPPORTED;
+  int rc = prepare_variant(dev, v);
+  if (rc) return rc;
+
+  const int KB = P.K / 128, NB = (P.N + 127) / 128;
+  const int m_ext = V.swap ? V.bnc : 128;
+  const int n_ext = V.swap ? 128 : V.bnc;
+  const int G_a = P.kind == kMasked ? P.G : 1;
+  const int G_b = P.kind == kDense ? 1 : P.G;
+
+  Params p{};
+  p.M = P.M;
+  p.N = P.N;
+  p.K = P.K;
+  p.KB = KB;
+  p.NB = NB;
+  p.G = G_b;
+  p.n_tiles = (P.N + n_ext - 1) / n_ext;
+  p.m_tiles = P.kind == kContiguous ? P.M / 128 : (P.M + m_ext - 1) / m_ext;
+  p.num_tiles = p.n_tiles * p.m_tiles * (P.kind == kMasked ? P.G : 1);
+  p.m_indices = P.kind == kContiguous ? P.idx : nullptr;
+  p.masked_m = P.kind == kMasked ? P.idx : nullptr;
+  p.sb = P.sb;
+  p.D = P.D;
+  if (p.num_tiles <= 0) return FP8G_OK;
+
+  CUtensorMap tmA, tmB, tmSA;
+  const uint32_t a_box_rows = V.swap ? V.bnc : 128;
+  const uint32_t b_box_rows = V.swap ? 128 : V.bnc;
+  rc = encode3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, P.A, P.K, P.M, G_a, (uint64_t)P.K,
+                (uint64_t)P.K * std::max(P.M, 1), 128, a_box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!rc)
+    rc = encode3d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, P.B, P.K, P.N, G_b, (uint64_t)P.K,
+                  (uint64_t)P.K * P.N, 128, b_box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!rc)
+    rc = encode3d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, P.sa, P.M, KB, G_a, (uint64_t)P.ld_sa * 4,
+                  (uint64_t)P.ld_sa * 4 * KB, V.swap ? V.bnc : 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = V.smem;
+  cfg.stream = stream;
+  if (V.split > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = V.split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(p.num_tiles * V.split, 1, 1);
+  } else {
+    cfg.gridDim = dim3(std::min(p.num_tiles, dev->sms), 1, 1);
+  }
+  void* args[] = {&tmA, &tmB, &tmSA, &p};
+  if (cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(V.fn), args) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FP8G_ERR_CUDA;
+  }
+  t_last_variant = v;
+  return FP8G_OK;
+}
+
+int select_variant(const Problem& P, DeviceInfo* dev) {
+  const int ov = g_override.load(std::memory_order_relaxed);
+  if (ov >= 0) return ov;
+  if (P.kind == kContiguous) return V_CONTIG_M128;
+  if (P.kind == kMasked) return P.expected_m > 0 && P.expected_m <= 64 ? V_MASKED_N64 : V_MASKED_N128;
+  if (P.M <= 64) {
+    const int nt = (P.N + 127) / 128;
+    if (P.K / 128 >= 16 && prepare_variant(dev, V_DENSE_SPLIT) == FP8G_OK &&
+        nt <= dev->max_clusters[V_DENSE_SPLIT] && nt * 8 <= dev->sms)
+      return V_DENSE_SPLIT;
+    return V_DENSE_N64;
+  }
+  return V_DENSE_M128;
+}
+
+int run(const Problem& P, cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const int v = select_variant(P, dev);
+  if (v < 0 || v >= kNumVariants) return FP8G_ERR_UNSUPPORTED;
+  return launch(P, v, dev, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8_gemm_nt(const uint8_t* A, const float* sa, int ld_sa, const uint8_t* B, const float* sb, uint16_t* D,
+                int M, int N, int K, cudaStream_t stream) {
+  int rc = check_shapes(M, N, K, ld_sa);
+  if (rc) return rc;
+  if (M == 0 || N == 0) return FP8G_OK;
+  if ((rc = check_ptrs(A, sa, B, sb, D))) return rc;
+  return run(Problem{kDense, A, sa, ld_sa, B, sb, D, nullptr, M, N, K, 1, 0}, stream);
+}
+
+int m_grouped_fp8_gemm_nt_contiguous(const uint8_t* A, const float* sa, int ld_sa, const uint8_t* B,
+                                     const float* sb, uint16_t* D, const int32_t* m_indices, int M, int N,
+                                     int K, int G, cudaStream_t stream) {
+  int rc = check_shapes(M, N, K, ld_sa);
+  if (rc) return rc;
+  if (G < 0 || M % 128 != 0) return FP8G_ERR_INVALID_ARG;
+  if (M == 0 || N == 0 || G == 0) return FP8G_OK;
+  if ((rc = check_ptrs(A, sa, B, sb, D))) return rc;
+  if (!m_indices) return FP8G_ERR_INVALID_ARG;
+  if (!aligned(m_indices, 4)) return FP8G_ERR_MISALIGNED;
+  return run(Problem{kContiguous, A, sa, ld_sa, B, sb, D, m_indices, M, N, K, G, 0}, stream);
+}
+
+int m_grouped_fp8_gemm_nt_masked(const uint8_t* A, const float* sa, int ld_sa, const uint8_t* B, const float* sb,
+                                 uint16_t* D, const int32_t* masked_m, int G, int Mmax, int N, int K,
+                                 int expected_m, cudaStream_t stream) {
+  int rc = check_shapes(Mmax, N, K, ld_sa);
+  if (rc) return rc;
+  if (G < 0 || expected_m < 0) return FP8G_ERR_INVALID_ARG;
+  if (Mmax == 0 || N == 0 || G == 0) return FP8G_OK;
+  if ((rc = check_ptrs(A, sa, B, sb, D))) return rc;
+  if (!masked_m) return FP8G_ERR_INVALID_ARG;
+  if (!aligned(masked_m, 4)) return FP8G_ERR_MISALIGNED;
+  return run(Problem{kMasked, A, sa, ld_sa, B, sb, D, masked_m, Mmax, N, K, G, expected_m}, stream);
+}
+
+const char* fp8g_status_string(int status) {
+  switch (status) {
+    case FP8G_OK: return "ok";
+    case FP8G_ERR_INVALID_ARG: return "invalid argument";
+    case FP8G_ERR_MISALIGNED: return "misaligned pointer or pitch";
+    case FP8G_ERR_UNSUPPORTED: return "unsupported device or no kernel variant for this call";
+    case FP8G_ERR_CUDA: return "CUDA call failed";
+    case FP8G_ERR_DEVICE: return "device-side error recorded";
+    default: return "unknown status";
+  }
+}
+
+int fp8g_get_device_error(int device, uint32_t* bits, int clear) {
+  int prev = 0;
+  if (cudaGetDevice(&prev) != cudaSuccess) return FP8G_ERR_CUDA;
+  if (device != prev && cudaSetDevice(device) != cudaSuccess) return FP8G_ERR_CUDA;
+  uint32_t w = 0;
+  int rc = FP8G_OK;
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpyFromSymbol(&w, g_fp8g_error_word, sizeof(w), 0, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    rc = FP8G_ERR_CUDA;
+  } else {
+    if (clear) {
+      const uint32_t z = 0;
+      if (cudaMemcpyToSymbol(g_fp8g_error_word, &z, sizeof(z), 0, cudaMemcpyHostToDevice) != cudaSuccess)
+        rc = FP8G_ERR_CUDA;
+    }
+    if (!rc && w) rc = FP8G_ERR_DEVICE;
+  }
+  if (bits) *bits = w;
+  if (device != prev) (void)cudaSetDevice(prev);
+  return rc;
+}
+
+int fp8g_set_variant_override(int variant) {
+  if (variant < -1 || variant >= kNumVariants) return FP8G_ERR_INVALID_ARG;
+  g_override.store(variant, std::memory_order_relaxed);
+  return FP8G_OK;
+}
+
+int fp8g_num_variants(void) { return kNumVariants; }
+
+const char* fp8g_variant_name(int variant) {
+  return variant >= 0 && variant < kNumVariants ? kVariants[variant].name : nullptr;
+}
+
+int fp8g_last_variant(void) { return t_last_variant; }
+
+int fp8g_version(void) { return 100; }
+
+}  // extern "C"

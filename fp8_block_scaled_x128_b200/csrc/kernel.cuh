@@ -1,0 +1,535 @@
+// kernel.cuh -- the fine-grained-scaled FP8 GEMM kernel for sm_100a.
+//
+//   D[m,n] = bf16( sum_kb P_kb[m,n] * sa[m,kb] * sb[n/128,kb] ),
+//   P_kb[m,n] = sum_{k in kb} A[m,k] * B[n,k]     (one 128-wide K-block)
+//
+// Fine-grained scaling of DeepSeek-V3 with the per-K-block partial promoted
+// out of the tensor-core accumulator onto the CUDA cores (GeekNews, "DeepSeek,
+// DeepGEMM 오픈소스 공개", topic body, first and fifth bullets).  The pages'
+// own design is a Hopper one (wgmma, register accumulators); this is a
+// Blackwell design:
+//
+//   warp 0        TMA producer: for every (tile, K-block) fills one stage of a
+//                 shared-memory ring with the 128-row "lane" operand tile,
+//                 the "column" operand tile and the tile's slice of sa.
+//   warp 1        MMA issuer (one thread): four tcgen05.mma kind::f8f6f4
+//                 (K = 32 each) write the K-block partial P_kb, FP32, into one
+//                 of several tensor-memory (TMEM) buffers; tcgen05.commit
+//                 frees the smem stage and signals the partial.
+//   warp 2        scale warp: turns the stage's sa slice and the tile's sb
+//                 row into the factors the promotion needs.
+//   warp 3        idle (completes warpgroup 0).
+//   warps 4..11   two promotion warpgroups, each owning half the tile's
+//                 columns: tcgen05.ld the finished partial, acc += P * scale
+//                 in FP32 registers (CUDA cores), release the TMEM buffer so
+//                 the MMA of a later K-block overlaps; after the tile's last
+//                 K-block, round to bf16 and store D.
+//
+// Orientation.  The MMA's M side (TMEM lanes) is always 128 rows.
+//   kSwap = true : lanes are 128 rows of B (n), columns are BNC rows of A
+//                  (m).  Used when M is small (decode), so that the large
+//                  operand fills the MMA's M; the B scale is one scalar per
+//                  (tile, K-block) and the A scale varies per column.
+//   kSwap = false: lanes are 128 rows of A (m), columns are BNC rows of B.
+//                  The A scale is one scalar per thread, the B scale one per
+//                  128 columns.
+// Scheduling kinds: dense; contiguous (128-row blocks of A map to experts via
+// m_indices, -1 = skip); masked (tiles at or past masked_m[g] are skipped).
+// SPLIT > 1 (dense, kSwap only): a cluster of SPLIT CTAs shares one output
+// tile, each over K/SPLIT, and the partial sums are reduced through
+// distributed shared memory in a fixed order (deterministic).
+//
+// Every wait is bounded: after kWaitTimeoutNs the waiter records
+// FP8G_DEVERR_TIMEOUT, raises a CTA-wide abort flag, and every role leaves
+// its loop; the teardown drains in-flight TMA and MMA work (again with a
+// bound) and frees TMEM before the CTA exits.
+#pragma once
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+#ifndef FP8G_DEVERR_TIMEOUT
+#define FP8G_DEVERR_TIMEOUT 0x1u
+#define FP8G_DEVERR_BAD_M_INDEX 0x2u
+#define FP8G_DEVERR_MASKED_OVER 0x4u
+#endif
+
+namespace fp8g {
+
+enum Kind : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+
+constexpr int kThreads = 384;
+constexpr int kKBMax = 512;                         // K <= 65536
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s
+constexpr uint64_t kDrainTimeoutNs = 100000000ull;  // 0.1 s
+
+// Per-device error word (FP8G_DEVERR_* bits); read by fp8g_get_device_error.
+__device__ uint32_t g_fp8g_error_word;
+
+struct Params {
+  int M;        // dense/contiguous: rows of A; masked: Mmax
+  int N, K, KB, NB, G;
+  int n_tiles;  // tiles along N
+  int m_tiles;  // tiles along M (per group for masked)
+  int num_tiles;
+  const int32_t* m_indices;
+  const int32_t* masked_m;
+  const float* sb;  // [G][NB][KB]
+  uint16_t* D;
+};
+
+constexpr int pow2_at_least(int x, int lo) {
+  int p = lo;
+  while (p < x) p *= 2;
+  return p;
+}
+
+template <bool kSwap, int BNC, int STAGES, int SPLIT>
+struct Layout {
+  static constexpr int kLaneBytes = 128 * 128;   // 128 rows x 128 e4m3 (one K-block)
+  static constexpr int kColBytes = BNC * 128;
+  static constexpr int kSaFloats = kSwap ? BNC : 128;  // sa slice: the tile's m-extent
+  static constexpr int kSclFloats = kSwap ? BNC : 4;   // scale factors per stage
+  static constexpr int kNBuf = BNC <= 128 ? 4 : 2;     // TMEM partial buffers
+  static constexpr int kTmemCols = pow2_at_least(kNBuf * BNC, 32);
+  static constexpr int kCW = BNC / 2;                  // columns per promotion warpgroup
+  static constexpr int kCPD = BNC / SPLIT;             // split-K: columns reduced per CTA
+  static constexpr int kOffLane = 0;
+  static constexpr int kOffCol = kOffLane + STAGES * kLaneBytes;
+  static constexpr int kOffSa = kOffCol + STAGES * kColBytes;
+  static constexpr int kOffScl = kOffSa + STAGES * kSaFloats * 4;
+  static constexpr int kOffSbRow = kOffScl + STAGES * kSclFloats * 4;
+  static constexpr int kOffRecv = kOffSbRow + 2 * kKBMax * 4;
+  static constexpr int kRecvBytes = SPLIT > 1 ? SPLIT * 128 * kCPD * 4 : 0;
+  static constexpr int kOffBar = kOffRecv + kRecvBytes;
+  static constexpr int kNumBars = 3 * STAGES + 2 * kNBuf + 2;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffMisc + 16;
+  static constexpr int kSmemAlloc = kBytes + 1024;  // + slack to align the base to 1024
+
+  static_assert(BNC % 32 == 0 && BNC >= 32 && BNC <= 256, "column tile");
+  static_assert(kCW % 32 == 0, "promotion chunking");
+  static_assert(kTmemCols <= 512, "TMEM");
+  static_assert(kOffCol % 1024 == 0 && kOffSa % 1024 == 0, "swizzle-128B tiles need 1024 alignment");
+  static_assert(kColBytes % 1024 == 0, "column tile rows must be a multiple of 8");
+  static_assert(SPLIT == 1 || (kSwap && BNC % SPLIT == 0 && kCW % kCPD == 0 && kCPD % 4 == 0),
+                "split-K layout");
+  static_assert(kSmemAlloc <= 232448, "shared memory");
+};
+
+struct Tile {
+  int g, m0, n0, mvalid, kb0, kb1;
+  bool valid;
+};
+
+// Tile t -> (group, rows, columns, valid row count, K-block range).  Every
+// role calls this with the same t and gets the same answer.
+template <bool kSwap, int BNC, int KIND, int SPLIT>
+__device__ __forceinline__ Tile get_tile(const Params& p, int t, uint32_t rank, bool report) {
+  constexpr int kMExt = kSwap ? BNC : 128;
+  constexpr int kNExt = kSwap ? 128 : BNC;
+  Tile T;
+  T.valid = true;
+  T.g = 0;
+  T.kb0 = 0;
+  T.kb1 = p.KB;
+  if constexpr (SPLIT > 1) {
+    T.kb0 = static_cast<int>((static_cast<long>(p.KB) * rank) / SPLIT);
+    T.kb1 = static_cast<int>((static_cast<long>(p.KB) * (rank + 1)) / SPLIT);
+  }
+  if constexpr (KIND == kDense) {
+    const int nt = t % p.n_tiles, mt = t / p.n_tiles;
+    T.m0 = mt * kMExt;
+    T.n0 = nt * kNExt;
+    T.mvalid = min(kMExt, p.M - T.m0);
+  } else if constexpr (KIND == kContiguous) {
+    const int nt = t % p.n_tiles, mt = t / p.n_tiles;
+    T.m0 = mt * 128;
+    T.n0 = nt * kNExt;
+    T.mvalid = 128;
+    const int g = __ldg(p.m_indices + mt);
+    if (g < 0 || g >= p.G) {
+      if (g >= p.G && report) atomicOr(&g_fp8g_error_word, FP8G_DEVERR_BAD_M_INDEX);
+      T.valid = false;
+    }
+    T.g = g;
+  } else {
+    const int per_g = p.n_tiles * p.m_tiles;
+    const int g = t / per_g, r = t % per_g;
+    const int nt = r / p.m_tiles, mt = r % p.m_tiles;  // tiles sharing a B tile are adjacent
+    int mg = __ldg(p.masked_m + g);
+    if (mg > p.M) {
+      if (report) atomicOr(&g_fp8g_error_word, FP8G_DEVERR_MASKED_OVER);
+      mg = p.M;
+    }
+    mg = max(mg, 0);
+    T.g = g;
+    T.m0 = mt * kMExt;
+    T.n0 = nt * kNExt;
+    T.mvalid = min(kMExt, mg - T.m0);
+    T.valid = T.m0 < mg;
+  }
+  return T;
+}
+
+// Bounded wait on a local mbarrier phase.  Returns false on timeout (after
+// recording it) or when another role has already aborted.
+template <bool kClusterScope = false>
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
+                                           volatile uint32_t* abort_flag) {
+  auto poll = [&]() {
+    return kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (poll()) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (poll()) return true;
+    if ((i & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        *abort_flag = 1u;
+        atomicOr(&g_fp8g_error_word, FP8G_DEVERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Teardown drain: like wait_phase, but ignores the abort flag and gives up
+// silently after kDrainTimeoutNs.
+__device__ __forceinline__ void drain_phase(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kDrainTimeoutNs) return;
+  }
+}
+
+template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT>
+__global__ void __launch_bounds__(kThreads, 1)
+    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmSA, const Params p) {
+  using L = Layout<kSwap, BNC, STAGES, SPLIT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  // barriers
+  const uint32_t bar0 = sbase + L::kOffBar;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto scl_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (3 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (3 * STAGES + L::kNBuf + b); };
+  const uint32_t recv_bar = bar0 + 8u * (3 * STAGES + 2 * L::kNBuf);
+  const uint32_t drain_bar = recv_bar + 8u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  // stage buffers
+  auto lane_tile = [&](int s) { return sbase + L::kOffLane + s * L::kLaneBytes; };
+  auto col_tile = [&](int s) { return sbase + L::kOffCol + s * L::kColBytes; };
+  auto sa_slice = [&](int s) { return sbase + L::kOffSa + s * L::kSaFloats * 4; };
+  float* sa_f = reinterpret_cast<float*>(smem + L::kOffSa);
+  float* scl_f = reinterpret_cast<float*>(smem + L::kOffScl);
+  float* sbrow = reinterpret_cast<float*>(smem + L::kOffSbRow);
+
+  constexpr int kPromoWarps = 8;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1 + kPromoWarps);
+      mbar_init(scl_bar(s), 1);
+    }
+    for (int b = 0; b < L::kNBuf; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), kPromoWarps);
+    }
+    mbar_init(recv_bar, SPLIT * 128);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmSA);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if constexpr (SPLIT > 1) cluster_sync_all();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const uint32_t rank = SPLIT > 1 ? cluster_ctarank() : 0u;
+  const int t_first = SPLIT > 1 ? static_cast<int>(blockIdx.x) / SPLIT : static_cast<int>(blockIdx.x);
+  const int t_step = SPLIT > 1 ? p.num_tiles : static_cast<int>(gridDim.x);
+  constexpr uint32_t kStageTx = L::kLaneBytes + L::kColBytes + L::kSaFloats * 4;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
+        const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t, rank, false);
+        if (!T.valid) continue;
+        const int ga = KIND == kMasked ? T.g : 0;
+        const int gb = KIND == kDense ? 0 : T.g;
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(s), kStageTx);
+          if constexpr (kSwap) {
+            tma_load_3d(lane_tile(s), &tmB, full_bar(s), kb * 128, T.n0, gb);
+            tma_load_3d(col_tile(s), &tmA, full_bar(s), kb * 128, T.m0, ga);
+          } else {
+            tma_load_3d(lane_tile(s), &tmA, full_bar(s), kb * 128, T.m0, ga);
+            tma_load_3d(col_tile(s), &tmB, full_bar(s), kb * 128, T.n0, gb);
+          }
+          tma_load_3d(sa_slice(s), &tmSA, full_bar(s), T.m0, kb, ga);
+        }
+      }
+      // drain: every issued load must land before the CTA may exit
+      const uint32_t first = it > static_cast<uint32_t>(STAGES) ? it - STAGES : 0u;
+      for (uint32_t i = first; i < it; ++i) drain_phase(full_bar(i % STAGES), (i / STAGES) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdesc = idesc_e4m3_f32(128, BNC);
+      uint32_t it = 0, tb = 0;
+      bool ok = true;
+      for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
+        const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t, rank, false);
+        if (!T.valid) continue;
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++it, ++tb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          const int b = tb % L::kNBuf;
+          const uint32_t tph = (tb / L::kNBuf) & 1u;
+          if (!wait_phase(full_bar(s), ph, abort_flag) ||
+              !wait_phase(tempty_bar(b), tph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BNC);
+          const uint64_t adesc = sdesc_k128_sw128(lane_tile(s));
+          const uint64_t bdesc = sdesc_k128_sw128(col_tile(s));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // 4 x K=32 bytes = one 128-wide K-block
+            mma_f8f6f4(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k),
+                       kIdesc, k > 0 ? 1u : 0u);
+          }
+          mma_commit(empty_bar(s));
+          mma_commit(tfull_bar(b));
+        }
+      }
+      // drain: all issued MMAs complete before TMEM is freed
+      mma_commit(drain_bar);
+      drain_phase(drain_bar, 0u);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale warp
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
+      const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t, rank, lane == 0);
+      if (!T.valid) continue;
+      // this tile's sb rows for its K-block range
+      constexpr int kRows = kSwap ? 1 : BNC / 128;
+      const int nkb = T.kb1 - T.kb0;
+      for (int j = 0; j < kRows; ++j) {
+        const int nb = T.n0 / 128 + j;
+        const float* src = p.sb + (static_cast<long>(T.g) * p.NB + nb) * p.KB + T.kb0;
+        for (int i = lane; i < nkb; i += 32) sbrow[j * kKBMax + i] = nb < p.NB ? __ldg(src + i) : 0.f;
+      }
+      __syncwarp();
+      for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        const bool w = wait_phase(full_bar(s), ph, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        if constexpr (kSwap) {
+          const float sbv = sbrow[kb - T.kb0];
+          const float* sa_s = sa_f + s * L::kSaFloats;
+          float* out = scl_f + s * L::kSclFloats;
+          for (int c = lane; c < BNC; c += 32) out[c] = sa_s[c] * sbv;
+        } else {
+          if (lane < kRows) scl_f[s * L::kSclFloats + lane] = sbrow[lane * kKBMax + (kb - T.kb0)];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(scl_bar(s));
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ promotion + epilogue
+    constexpr int kCW = L::kCW;
+    const int wg = (warp - 4) / 4;  // column half
+    const int q = warp % 4;         // TMEM lane quarter this warp may access
+    const int row = 32 * q + lane;  // tile row = TMEM lane
+    float acc[kCW];
+    uint32_t it = 0, tb = 0;
+    bool ok = true;
+    for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
+      const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t, rank, false);
+      if (!T.valid) continue;
+#pragma unroll
+      for (int c = 0; c < kCW; ++c) acc[c] = 0.f;
+      // column chunks of 32 that hold valid output (kSwap: columns are rows of A)
+      const int live = kSwap ? min(kCW, max(0, T.mvalid - wg * kCW)) : kCW;
+      for (int kb = T.kb0; kb < T.kb1; ++kb, ++it, ++tb) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        const int b = tb % L::kNBuf;
+        const uint32_t tph = (tb / L::kNBuf) & 1u;
+        bool w = wait_phase(tfull_bar(b), tph, abort_flag);
+        w = w && wait_phase(scl_bar(s), ph, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                               static_cast<uint32_t>(b * BNC + wg * kCW);
+        uint32_t r[kCW / 32][32];
+#pragma unroll
+        for (int j = 0; j < kCW / 32; ++j)
+          if (32 * j < live) tmem_ld_32x32b_x32(taddr + 32 * j, r[j]);
+        tmem_ld_wait_bind(r[0]);
+#pragma unroll
+        for (int j = 1; j < kCW / 32; ++j) bind_after_wait(r[j]);
+        if constexpr (kSwap) {
+          const float4* f4 = reinterpret_cast<const float4*>(scl_f + s * L::kSclFloats + wg * kCW);
+#pragma unroll
+          for (int j = 0; j < kCW / 32; ++j) {
+            if (32 * j < live) {
+#pragma unroll
+              for (int c4 = 0; c4 < 8; ++c4) {
+                const float4 f = f4[8 * j + c4];
+                float* a = acc + 32 * j + 4 * c4;
+                a[0] = fmaf(__uint_as_float(r[j][4 * c4 + 0]), f.x, a[0]);
+                a[1] = fmaf(__uint_as_float(r[j][4 * c4 + 1]), f.y, a[1]);
+                a[2] = fmaf(__uint_as_float(r[j][4 * c4 + 2]), f.z, a[2]);
+                a[3] = fmaf(__uint_as_float(r[j][4 * c4 + 3]), f.w, a[3]);
+              }
+            }
+          }
+        } else {
+          const float sc = sa_f[s * L::kSaFloats + row] * scl_f[s * L::kSclFloats + (wg * kCW) / 128];
+#pragma unroll
+          for (int j = 0; j < kCW / 32; ++j)
+#pragma unroll
+            for (int c = 0; c < 32; ++c) acc[32 * j + c] = fmaf(__uint_as_float(r[j][c]), sc, acc[32 * j + c]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(tempty_bar(b));
+          mbar_arrive(empty_bar(s));
+        }
+      }
+      if (!ok) break;
+
+      const long drow0 = KIND == kMasked ? static_cast<long>(T.g) * p.M : 0;
+      if constexpr (SPLIT > 1) {
+        // push this CTA's partial columns to the CTA that reduces them
+        constexpr int kCPD = L::kCPD;
+        const uint32_t recv_local = sbase + L::kOffRecv + (rank * 128u + row) * (kCPD * 4u);
+#pragma unroll
+        for (int d0 = 0; d0 < kCW; d0 += kCPD) {
+          const uint32_t dst = static_cast<uint32_t>((wg * kCW + d0) / kCPD);
+          const uint32_t raddr = mapa(recv_local, dst);
+#pragma unroll
+          for (int c = 0; c < kCPD; c += 4)
+            st_cluster_v4(raddr + 4u * c, acc[d0 + c], acc[d0 + c + 1], acc[d0 + c + 2], acc[d0 + c + 3]);
+          mbar_arrive_remote(mapa(recv_bar, dst));
+        }
+        // reduce the columns this CTA owns, in source-rank order
+        if (wg == static_cast<int>((rank * kCPD) / kCW)) {
+          const bool w = wait_phase<true>(recv_bar, 0u, abort_flag);
+          if (!__all_sync(0xffffffffu, w)) {
+            ok = false;
+            break;
+          }
+          float sum[kCPD];
+#pragma unroll
+          for (int c = 0; c < kCPD; ++c) sum[c] = 0.f;
+          const float* rv = reinterpret_cast<const float*>(smem + L::kOffRecv);
+          for (int src = 0; src < SPLIT; ++src) {
+            const float4* v = reinterpret_cast<const float4*>(rv + (src * 128 + row) * kCPD);
+#pragma unroll
+            for (int c4 = 0; c4 < kCPD / 4; ++c4) {
+              const float4 f = v[c4];
+              sum[4 * c4 + 0] += f.x;
+              sum[4 * c4 + 1] += f.y;
+              sum[4 * c4 + 2] += f.z;
+              sum[4 * c4 + 3] += f.w;
+            }
+          }
+          const int n = T.n0 + row;
+          if (n < p.N) {
+#pragma unroll
+            for (int c = 0; c < kCPD; ++c) {
+              const int mc = static_cast<int>(rank) * kCPD + c;
+              if (mc < T.mvalid)
+                p.D[(drow0 + T.m0 + mc) * p.N + n] = static_cast<uint16_t>(pack_bf16x2(sum[c], 0.f) & 0xFFFFu);
+            }
+          }
+        }
+      } else if constexpr (kSwap) {
+        // lanes hold consecutive n: each column store is 64 contiguous bytes per warp
+        const int n = T.n0 + row;
+        if (n < p.N) {
+          uint16_t* dcol = p.D + (drow0 + T.m0 + wg * kCW) * p.N + n;
+#pragma unroll
+          for (int c = 0; c < kCW; ++c)
+            if (c < live) dcol[static_cast<long>(c) * p.N] = static_cast<uint16_t>(pack_bf16x2(acc[c], 0.f) & 0xFFFFu);
+        }
+      } else {
+        // a thread holds kCW consecutive columns of its row: 16-byte stores
+        if (row < T.mvalid) {
+          uint16_t* drow = p.D + (drow0 + T.m0 + row) * p.N + T.n0 + wg * kCW;
+#pragma unroll
+          for (int c = 0; c < kCW; c += 8) {
+            if (T.n0 + wg * kCW + c < p.N) {
+              uint4 v;
+              v.x = pack_bf16x2(acc[c + 0], acc[c + 1]);
+              v.y = pack_bf16x2(acc[c + 2], acc[c + 3]);
+              v.z = pack_bf16x2(acc[c + 4], acc[c + 5]);
+              v.w = pack_bf16x2(acc[c + 6], acc[c + 7]);
+              *reinterpret_cast<uint4*>(drow + c) = v;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+  if constexpr (SPLIT > 1) cluster_sync_all();  // no CTA leaves while a peer may still write to it
+}
+
+}  // namespace fp8g

@@ -1,0 +1,141 @@
+"""Python binding of the C ABI in include/fp8gemm.h (ctypes; marshalling only).
+
+Every function takes torch CUDA tensors in the library's layouts, passes their
+device pointers and the current CUDA stream to libfp8gemm.so, and raises if the
+library returns an error.  No step of the GEMM runs in Python or on the CPU; if
+the shared library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8gemm.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m fp8_block_scaled_x128_b200.build` "
+        "(the library has no CPU fallback)")
+
+_P, _I, _U32 = C.c_void_p, C.c_int, C.c_uint32
+
+lib = C.CDLL(LIB_PATH)
+lib.fp8_gemm_nt.restype = _I
+lib.fp8_gemm_nt.argtypes = [_P, _P, _I, _P, _P, _P, _I, _I, _I, _P]
+lib.m_grouped_fp8_gemm_nt_contiguous.restype = _I
+lib.m_grouped_fp8_gemm_nt_contiguous.argtypes = [_P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P]
+lib.m_grouped_fp8_gemm_nt_masked.restype = _I
+lib.m_grouped_fp8_gemm_nt_masked.argtypes = [_P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
+lib.fp8g_status_string.restype = C.c_char_p
+lib.fp8g_status_string.argtypes = [_I]
+lib.fp8g_get_device_error.restype = _I
+lib.fp8g_get_device_error.argtypes = [_I, C.POINTER(_U32), _I]
+lib.fp8g_set_variant_override.restype = _I
+lib.fp8g_set_variant_override.argtypes = [_I]
+lib.fp8g_num_variants.restype = _I
+lib.fp8g_num_variants.argtypes = []
+lib.fp8g_variant_name.restype = C.c_char_p
+lib.fp8g_variant_name.argtypes = [_I]
+lib.fp8g_last_variant.restype = _I
+lib.fp8g_last_variant.argtypes = []
+lib.fp8g_version.restype = _I
+lib.fp8g_version.argtypes = []
+
+DEVERR_TIMEOUT, DEVERR_BAD_M_INDEX, DEVERR_MASKED_OVER = 0x1, 0x2, 0x4
+
+
+class Fp8GemmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib.fp8g_status_string(status).decode()} (status {status})")
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise Fp8GemmError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _dev(t, dt, name):
+    if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
+        raise TypeError(f"{name}: expected a contiguous CUDA tensor of {dt}, got {t.dtype} on {t.device}")
+    return t
+
+
+def variant_names():
+    return [lib.fp8g_variant_name(i).decode() for i in range(lib.fp8g_num_variants())]
+
+
+def set_variant_override(v: int | None) -> None:
+    _check(lib.fp8g_set_variant_override(-1 if v is None else int(v)), "fp8g_set_variant_override")
+
+
+def last_variant() -> int:
+    return lib.fp8g_last_variant()
+
+
+def device_error(clear: bool = True, device: int | None = None) -> int:
+    """The device error word (FP8G_DEVERR_* bits); synchronises the device."""
+    bits = _U32(0)
+    d = torch.cuda.current_device() if device is None else device
+    rc = lib.fp8g_get_device_error(int(d), C.byref(bits), int(clear))
+    if rc not in (0, 5):
+        raise Fp8GemmError(rc, "fp8g_get_device_error")
+    return bits.value
+
+
+def fp8_gemm_nt(A, sa, B, sb, D=None, stream=None):
+    """Dense: A [M,K] uint8 (e4m3 codes), sa [K/128, ld_sa] float32, B [N,K] uint8,
+    sb [ceil(N/128), K/128] float32 -> D [M,N] bfloat16."""
+    M, K = A.shape
+    N = B.shape[0]
+    _dev(A, torch.uint8, "A"), _dev(B, torch.uint8, "B")
+    _dev(sa, torch.float32, "sa"), _dev(sb, torch.float32, "sb")
+    if D is None:
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _dev(D, torch.bfloat16, "D")
+    _check(lib.fp8_gemm_nt(_ptr(A), _ptr(sa), sa.shape[1], _ptr(B), _ptr(sb), _ptr(D), M, N, K,
+                           _stream(stream)), "fp8_gemm_nt")
+    return D
+
+
+def m_grouped_fp8_gemm_nt_contiguous(A, sa, B, sb, m_indices, D=None, stream=None):
+    """Contiguous: A [M,K], sa [K/128, ld_sa], B [G,N,K], sb [G, ceil(N/128), K/128],
+    m_indices [M/128] int32 -> D [M,N] bfloat16 (rows of -1 blocks untouched)."""
+    M, K = A.shape
+    G, N, _ = B.shape
+    _dev(A, torch.uint8, "A"), _dev(B, torch.uint8, "B"), _dev(m_indices, torch.int32, "m_indices")
+    _dev(sa, torch.float32, "sa"), _dev(sb, torch.float32, "sb")
+    if D is None:
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _dev(D, torch.bfloat16, "D")
+    _check(lib.m_grouped_fp8_gemm_nt_contiguous(_ptr(A), _ptr(sa), sa.shape[1], _ptr(B), _ptr(sb), _ptr(D),
+                                                _ptr(m_indices), M, N, K, G, _stream(stream)),
+           "m_grouped_fp8_gemm_nt_contiguous")
+    return D
+
+
+def m_grouped_fp8_gemm_nt_masked(A, sa, B, sb, masked_m, expected_m, D=None, stream=None):
+    """Masked: A [G,Mmax,K], sa [G, K/128, ld_sa], B [G,N,K], sb [G, ceil(N/128), K/128],
+    masked_m [G] int32 (device) -> D [G,Mmax,N] bfloat16 (rows >= masked_m[g] untouched)."""
+    G, Mmax, K = A.shape
+    N = B.shape[1]
+    _dev(A, torch.uint8, "A"), _dev(B, torch.uint8, "B"), _dev(masked_m, torch.int32, "masked_m")
+    _dev(sa, torch.float32, "sa"), _dev(sb, torch.float32, "sb")
+    if D is None:
+        D = torch.empty((G, Mmax, N), dtype=torch.bfloat16, device=A.device)
+    _dev(D, torch.bfloat16, "D")
+    _check(lib.m_grouped_fp8_gemm_nt_masked(_ptr(A), _ptr(sa), sa.shape[2], _ptr(B), _ptr(sb), _ptr(D),
+                                            _ptr(masked_m), G, Mmax, N, K, int(expected_m),
+                                            _stream(stream)), "m_grouped_fp8_gemm_nt_masked")
+    return D

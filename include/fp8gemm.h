@@ -1,0 +1,151 @@
+/*
+ * fp8gemm.h -- C ABI of the fine-grained-scaled FP8 GEMM library for B200
+ * (sm_100a).
+ *
+ * The operation (all three entry points):
+ *
+ *   D[m,n] = bf16_rne( sum_{kb} ( sum_{k = 128kb}^{128kb+127} A[m,k] * B[n,k] )
+ *                               * sa[m,kb] * sb[n/128,kb] )
+ *
+ * A and B are FP8 e4m3 ("fn": bias 7, no infinities, max 448).  A carries one
+ * FP32 scale per 1x128 group of a row; B carries one FP32 scale per 128x128
+ * block.  This is the fine-grained scaling of DeepSeek-V3 (GeekNews, "DeepSeek,
+ * DeepGEMM 오픈소스 공개", topic body, first bullet).  Each 128-wide K-block
+ * partial is formed by the tensor cores and then promoted to an FP32
+ * accumulator on the CUDA cores (same page, fifth bullet).  "NT": both operands
+ * are K-major, so B is the transposed weight, and converting and transposing
+ * inputs is the caller's job (kakushin.no, "Hvorfor FP8 og FP4 er
+ * interessant").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers on the current device.  They are
+ *    owned by the caller; the library neither allocates nor frees them.
+ *  - Layouts are dense and row-major:
+ *      A  [M, K] uint8 e4m3 codes, row pitch K bytes
+ *      B  [N, K] uint8 e4m3 codes, row pitch K bytes
+ *      sa [KB][ld_sa] float: sa[kb*ld_sa + m] scales A[m, 128kb .. 128kb+127]
+ *         ("MN-major": one K-block's scales for consecutive rows are adjacent)
+ *      sb [NB][KB] float: sb[nb*KB + kb] scales B[128nb .. +127, 128kb .. +127]
+ *      D  [M, N] bf16 (bit patterns), row pitch N elements
+ *    where KB = K/128 and NB = ceil(N/128).  If N % 128 != 0, the last scale
+ *    block covers the remaining N % 128 rows.
+ *  - Requirements (otherwise FP8G_ERR_INVALID_ARG / FP8G_ERR_MISALIGNED):
+ *      K > 0, K % 128 == 0, K <= 65536; M, N >= 0; N % 8 == 0;
+ *      ld_sa >= M (Mmax for the masked call) and ld_sa % 4 == 0;
+ *      A, B, sa, D 16-byte aligned; sb, m_indices, masked_m 4-byte aligned.
+ *    M == 0 or N == 0 (or G == 0) is a no-op that returns FP8G_OK.
+ *  - The call enqueues kernels on `stream` and returns without waiting.  It
+ *    never synchronises and never reads device memory on the host, so it can
+ *    be captured in a CUDA graph.  D is complete when the stream reaches
+ *    that point.
+ *  - Errors found on the host come back as the return value; nothing is
+ *    launched then.  Errors found by the kernel (a bad m_indices entry, a
+ *    masked_m above Mmax, a pipeline wait that timed out) are recorded in a
+ *    per-device error word.  Read it with fp8g_get_device_error().
+ *  - The calls are thread-safe with respect to one another.
+ *  - Needs a compute capability 10.0 device (B200); otherwise
+ *    FP8G_ERR_UNSUPPORTED.
+ */
+#ifndef FP8GEMM_H
+#define FP8GEMM_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum fp8g_status {
+    FP8G_OK = 0,
+    FP8G_ERR_INVALID_ARG = 1,   /* null pointer, bad size, K % 128 != 0, ... */
+    FP8G_ERR_MISALIGNED = 2,    /* pointer or pitch alignment not met */
+    FP8G_ERR_UNSUPPORTED = 3,   /* device is not sm_100, or no kernel variant fits */
+    FP8G_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (launch, attribute, ...) */
+    FP8G_ERR_DEVICE = 5         /* fp8g_get_device_error found a recorded device-side error */
+};
+
+/* Device-side error word bits (fp8g_get_device_error). */
+#define FP8G_DEVERR_TIMEOUT       0x1u  /* a pipeline wait gave up; outputs of that call are invalid */
+#define FP8G_DEVERR_BAD_M_INDEX   0x2u  /* contiguous: m_indices entry >= G (block skipped) */
+#define FP8G_DEVERR_MASKED_OVER   0x4u  /* masked: masked_m[g] > Mmax (clamped to Mmax) */
+
+/*
+ * Dense NT GEMM (GeekNews page, "일반 GEMM 성능 (Dense 모델)").
+ *   A [M,K], sa [K/128][ld_sa], B [N,K], sb [ceil(N/128)][K/128], D [M,N].
+ * Every element of D is written.
+ */
+int fp8_gemm_nt(const uint8_t *A, const float *sa, int ld_sa,
+                const uint8_t *B, const float *sb,
+                uint16_t *D, int M, int N, int K, cudaStream_t stream);
+
+/*
+ * M-grouped contiguous GEMM for MoE prefill/training (GeekNews page,
+ * "연속된(contiguous) 레이아웃의 그룹화 GEMM": rows grouped along M, N and K shared).
+ * The experts' row segments are concatenated along M.  Each segment is padded
+ * to a multiple of 128 rows, so every 128-row block belongs to one expert.
+ *   A [M,K] with M % 128 == 0, sa [K/128][ld_sa],
+ *   B [G,N,K], sb [G][ceil(N/128)][K/128], D [M,N],
+ *   m_indices [M/128] int32 (device): expert of each 128-row block.  -1 means
+ *   the block belongs to no expert; its D rows are left untouched.  Padding
+ *   rows inside a block are computed with that block's expert.
+ */
+int m_grouped_fp8_gemm_nt_contiguous(const uint8_t *A, const float *sa, int ld_sa,
+                                     const uint8_t *B, const float *sb, uint16_t *D,
+                                     const int32_t *m_indices,
+                                     int M, int N, int K, int G, cudaStream_t stream);
+
+/*
+ * M-grouped masked GEMM for MoE decode under CUDA graphs (GeekNews page,
+ * "마스킹(masked) 레이아웃의 그룹화 GEMM": the host does not know how many
+ * tokens each expert got, so a mask tensor tells the kernel how much work to
+ * do).
+ *   A [G,Mmax,K], sa [G][K/128][ld_sa], B [G,N,K], sb [G][ceil(N/128)][K/128],
+ *   D [G,Mmax,N], masked_m [G] int32 (device, never read on the host).
+ * Group g computes its first min(masked_m[g], Mmax) rows; rows at and beyond
+ * that count are left untouched.  expected_m is a hint (the typical
+ * masked_m) used only to pick a kernel variant; results do not depend on it.
+ */
+int m_grouped_fp8_gemm_nt_masked(const uint8_t *A, const float *sa, int ld_sa,
+                                 const uint8_t *B, const float *sb, uint16_t *D,
+                                 const int32_t *masked_m,
+                                 int G, int Mmax, int N, int K, int expected_m,
+                                 cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char *fp8g_status_string(int status);
+
+/*
+ * Reads this library's device-side error word on `device` into *bits (the
+ * FP8G_DEVERR_* flags of every call since the last clear).  If `clear` is
+ * nonzero, it also resets the word.  Synchronises the device.  Returns
+ * FP8G_OK if the word is zero, FP8G_ERR_DEVICE if it is not, and
+ * FP8G_ERR_CUDA if the read itself failed.
+ */
+int fp8g_get_device_error(int device, uint32_t *bits, int clear);
+
+/*
+ * Tuning and testing: force the kernel variant that the next calls use.
+ * Pass -1 to restore automatic selection.  Variants are listed by
+ * fp8g_variant_name(i) for i = 0 .. fp8g_num_variants()-1.  A forced variant
+ * that cannot run a given call makes that call return FP8G_ERR_UNSUPPORTED.
+ * The setting is process-wide.
+ */
+int fp8g_set_variant_override(int variant);
+int fp8g_num_variants(void);
+const char *fp8g_variant_name(int variant);
+
+/*
+ * The variant that the last successful call on this thread launched, or -1.
+ */
+int fp8g_last_variant(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int fp8g_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8GEMM_H */

@@ -1,0 +1,115 @@
+"""The C-ABI library on a machine without a GPU: it builds for sm_100a, loads,
+exports every entry point declared in include/fp8gemm.h, and rejects bad
+arguments on the host before touching the device."""
+import ctypes as C
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8gemm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp8_block_scaled_x128_b200 import build
+    path = build.build()
+    L = C.CDLL(path)
+    P, I = C.c_void_p, C.c_int
+    L.fp8_gemm_nt.argtypes = [P, P, I, P, P, P, I, I, I, P]
+    L.m_grouped_fp8_gemm_nt_contiguous.argtypes = [P, P, I, P, P, P, P, I, I, I, I, P]
+    L.m_grouped_fp8_gemm_nt_masked.argtypes = [P, P, I, P, P, P, P, I, I, I, I, I, P]
+    L.fp8g_status_string.restype = C.c_char_p
+    L.fp8g_variant_name.restype = C.c_char_p
+    return L
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_three_entry_points():
+    names = declared_functions()
+    for n in ("fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_library_is_built_for_sm100a():
+    from fp8_block_scaled_x128_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.FLAGS)
+
+
+# fake, never-dereferenced device addresses: every call below returns before any CUDA call
+A = B = D = 0x7f0000000000
+SA = SB = 0x7f0000100000
+S = None
+
+
+@pytest.mark.parametrize("args,status", [
+    ((A, SA, 64, B, SB, D, 64, 2112, 100, S), 1),      # K not a multiple of 128
+    ((A, SA, 64, B, SB, D, 64, 2112, 0, S), 1),        # K == 0
+    ((A, SA, 64, B, SB, D, 64, 2112, 128 * 513, S), 1),  # K too large
+    ((A, SA, 64, B, SB, D, -1, 2112, 128, S), 1),      # negative M
+    ((A, SA, 32, B, SB, D, 64, 2112, 128, S), 1),      # ld_sa < M
+    ((A, SA, 64, B, SB, D, 64, 2110, 128, S), 2),      # N % 8 != 0
+    ((A, SA, 66, B, SB, D, 64, 2112, 128, S), 2),      # ld_sa % 4 != 0
+    ((None, SA, 64, B, SB, D, 64, 2112, 128, S), 1),   # null A
+    ((A, SA, 64, B, None, D, 64, 2112, 128, S), 1),    # null sb
+    ((A + 8, SA, 64, B, SB, D, 64, 2112, 128, S), 2),  # A not 16-byte aligned
+    ((A, SA, 64, B, SB, D + 2, 64, 2112, 128, S), 2),  # D not 16-byte aligned
+    ((A, SA + 4, 64, B, SB, D, 64, 2112, 128, S), 2),  # sa not 16-byte aligned
+    ((A, SA, 64, B, SB + 2, D, 64, 2112, 128, S), 2),  # sb not 4-byte aligned
+    ((None, None, 4, None, None, None, 0, 2112, 128, S), 0),  # M == 0: no-op
+    ((None, None, 64, None, None, None, 64, 0, 128, S), 0),   # N == 0: no-op
+])
+def test_dense_host_validation(lib, args, status):
+    assert lib.fp8_gemm_nt(*args) == status
+
+
+def test_contiguous_host_validation(lib):
+    f = lib.m_grouped_fp8_gemm_nt_contiguous
+    idx = 0x7f0000200000
+    assert f(A, SA, 256, B, SB, D, idx, 200, 128, 128, 2, S) == 1       # M % 128 != 0
+    assert f(A, SA, 256, B, SB, D, None, 256, 128, 128, 2, S) == 1      # null m_indices
+    assert f(A, SA, 256, B, SB, D, idx + 2, 256, 128, 128, 2, S) == 2   # misaligned m_indices
+    assert f(A, SA, 256, B, SB, D, idx, 256, 128, 128, -1, S) == 1      # G < 0
+    assert f(None, None, 4, None, None, None, None, 0, 128, 128, 2, S) == 0
+
+
+def test_masked_host_validation(lib):
+    f = lib.m_grouped_fp8_gemm_nt_masked
+    mm = 0x7f0000200000
+    assert f(A, SA, 256, B, SB, D, None, 4, 256, 128, 128, 128, S) == 1   # null masked_m
+    assert f(A, SA, 252, B, SB, D, mm, 4, 256, 128, 128, 128, S) == 1     # ld_sa < Mmax
+    assert f(A, SA, 256, B, SB, D, mm, 4, 256, 128, 128, -1, S) == 1      # expected_m < 0
+    assert f(A, SA, 256, B, SB, D, mm, 4, 256, 130, 128, 128, S) == 2     # N % 8
+    assert f(None, None, 256, None, None, None, None, 0, 256, 128, 128, 1, S) == 0  # G == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_valid_call_without_gpu_reports_cuda_error(lib):
+    assert lib.fp8_gemm_nt(A, SA, 64, B, SB, D, 64, 2112, 7168, S) == 4
+
+
+def test_status_strings_and_variant_table(lib):
+    for s in range(6):
+        assert lib.fp8g_status_string(s)
+    n = lib.fp8g_num_variants()
+    assert n >= 3
+    names = [lib.fp8g_variant_name(i).decode() for i in range(n)]
+    assert len(set(names)) == n
+    assert lib.fp8g_variant_name(n) is None
+    assert lib.fp8g_set_variant_override(n) == 1
+    assert lib.fp8g_set_variant_override(-2) == 1
+    assert lib.fp8g_set_variant_override(0) == 0
+    assert lib.fp8g_set_variant_override(-1) == 0
+    assert lib.fp8g_version() >= 100

@@ -1,0 +1,309 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Inputs come from the seeded generator; expected values come from the oracle
+only.  Floating-point cases use the acceptance tolerance of parity_util;
+exact-integer cases (codes in {-2..2}, power-of-two scales) must match the
+oracle's bf16 bits exactly.  Rows that the method must not write (masked rows
+past masked_m, contiguous blocks marked -1) are checked bit-for-bit against
+a canary fill.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_block_scaled_x128_b200 import synth
+
+from .parity_util import CANARY, assert_close, exact_integer_codes, pow2_scales
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def g():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from fp8_block_scaled_x128_b200 import gemm
+    gemm.device_error(clear=True)
+    yield gemm
+    gemm.set_variant_override(None)
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host_bits(t):
+    torch.cuda.synchronize()
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def canary_like(shape):
+    return torch.full(shape, CANARY - 0x10000, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+
+
+def variants(g, prefix):
+    return [i for i, n in enumerate(g.variant_names()) if n.startswith(prefix)]
+
+
+def dense_gpu(g, d, variant=None):
+    g.set_variant_override(variant)
+    try:
+        D = g.fp8_gemm_nt(dev(d["A"]), dev(d["sa"]), dev(d["B"]), dev(d["sb"]))
+        if variant is not None:
+            assert g.last_variant() == variant
+        return host_bits(D)
+    finally:
+        g.set_variant_override(None)
+
+
+def exact_dense(seed, M, N, K):
+    rng = np.random.default_rng(seed)
+    KB, NB = K // 128, (N + 127) // 128
+    ld = synth.ld_for(M)
+    sa = np.zeros((KB, ld), np.float32)
+    sa[:, :M] = pow2_scales(rng, (KB, M))
+    return dict(A=exact_integer_codes(rng, (M, K)), sa=sa, ld_sa=ld, B=exact_integer_codes(rng, (N, K)),
+                sb=pow2_scales(rng, (NB, KB)), M=M, N=N, K=K)
+
+
+def oracle_dense(d, rows=None):
+    return oracle.gemm_nt(d["A"], d["sa"], d["ld_sa"], d["B"], d["sb"], d["M"], d["N"], d["K"], rows=rows)
+
+
+# --------------------------------------------------------------------------- dense
+
+DENSE_SHAPES = [(1, 8, 128), (64, 256, 384), (65, 200, 256), (128, 256, 512), (200, 136, 1024),
+                (257, 520, 256), (64, 2112, 2048)]
+
+
+@pytest.mark.parametrize("shape", DENSE_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_dense_every_variant(g, shape):
+    M, N, K = shape
+    d = synth.dense_inputs(100 + M + N, M, N, K)
+    ex, _ = oracle_dense(d)
+    for v in variants(g, "dense_"):
+        assert_close(dense_gpu(g, d, v), ex, f"{g.variant_names()[v]} {shape}")
+    assert g.device_error() == 0
+
+
+@pytest.mark.parametrize("shape", [(64, 256, 1024), (130, 264, 512), (64, 2112, 7168)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_dense_exact_integers_bit_exact(g, shape):
+    d = exact_dense(7, *shape)
+    _, bf = oracle_dense(d)
+    for v in variants(g, "dense_"):
+        got = dense_gpu(g, d, v)
+        assert np.array_equal(got, bf), g.variant_names()[v]
+
+
+def test_dense_config_128x256x512(g):
+    d = synth.config_inputs("dense_128x256x512")
+    ex, _ = oracle_dense(d)
+    assert_close(dense_gpu(g, d), ex, "dense_128x256x512")
+
+
+def test_dense_config_64x2112x7168_all_variants(g):
+    d = synth.config_inputs("dense_64x2112x7168")
+    ex, _ = oracle_dense(d)
+    assert_close(dense_gpu(g, d), ex, "auto")
+    for v in variants(g, "dense_"):
+        assert_close(dense_gpu(g, d, v), ex, g.variant_names()[v])
+
+
+def test_dense_is_deterministic(g):
+    d = synth.config_inputs("dense_64x2112x7168")
+    first = dense_gpu(g, d)
+    for _ in range(3):
+        assert np.array_equal(dense_gpu(g, d), first)
+
+
+# --------------------------------------------------------------------------- contiguous
+
+def contig_gpu(g, d, variant=None):
+    g.set_variant_override(variant)
+    try:
+        D = canary_like((d["M"], d["N"]))
+        g.m_grouped_fp8_gemm_nt_contiguous(dev(d["A"]), dev(d["sa"]), dev(d["B"]), dev(d["sb"]),
+                                           dev(d["m_indices"]), D=D)
+        if variant is not None:
+            assert g.last_variant() == variant
+        return host_bits(D)
+    finally:
+        g.set_variant_override(None)
+
+
+def check_contig(g, d, exact=False):
+    M, N = d["M"], d["N"]
+    ex, bf = oracle.m_grouped_contiguous(d["A"], d["sa"], d["ld_sa"], d["B"], d["sb"], d["m_indices"],
+                                         M, N, d["K"], d["G"])
+    live = np.repeat(d["m_indices"] >= 0, 128)
+    for v in variants(g, "contiguous_"):
+        got = contig_gpu(g, d, v)
+        name = g.variant_names()[v]
+        assert np.all(got[~live] == CANARY), f"{name}: skipped block written"
+        if exact:
+            assert np.array_equal(got[live], bf[live]), name
+        else:
+            assert_close(got[live], ex[live], name)
+
+
+def test_contiguous_ragged_experts_and_skipped_blocks(g):
+    d = synth.contiguous_inputs(21, [100, 256, 20, 300], 136, 512, empty_blocks=(1, 5))
+    check_contig(g, d)
+    assert g.device_error() == 0
+
+
+def test_contiguous_exact_integers(g):
+    d = synth.contiguous_inputs(22, [128, 200, 64], 264, 384, empty_blocks=(2,))
+    rng = np.random.default_rng(5)
+    d["A"] = exact_integer_codes(rng, d["A"].shape)
+    d["B"] = exact_integer_codes(rng, d["B"].shape)
+    d["sa"][:, :d["M"]] = pow2_scales(rng, (d["K"] // 128, d["M"]))
+    d["sb"] = pow2_scales(rng, d["sb"].shape)
+    check_contig(g, d, exact=True)
+
+
+def test_contiguous_bad_expert_index_is_flagged_and_skipped(g):
+    d = synth.contiguous_inputs(23, [128, 128], 64, 128)
+    d["m_indices"] = np.array([0, 7], np.int32)  # 7 >= G
+    g.device_error(clear=True)
+    got = contig_gpu(g, d)
+    assert np.all(got[128:] == CANARY)
+    assert g.device_error() & g.DEVERR_BAD_M_INDEX
+
+
+# --------------------------------------------------------------------------- masked
+
+def masked_gpu(g, d, variant=None, expected_m=None):
+    g.set_variant_override(variant)
+    try:
+        D = canary_like((d["G"], d["Mmax"], d["N"]))
+        g.m_grouped_fp8_gemm_nt_masked(dev(d["A"]), dev(d["sa"]), dev(d["B"]), dev(d["sb"]),
+                                       dev(d["masked_m"]), d["Mmax"] // 2 if expected_m is None else expected_m,
+                                       D=D)
+        if variant is not None:
+            assert g.last_variant() == variant
+        return host_bits(D)
+    finally:
+        g.set_variant_override(None)
+
+
+def check_masked(g, d, exact=False):
+    G, Mmax, N, K = d["G"], d["Mmax"], d["N"], d["K"]
+    ex, bf = oracle.m_grouped_masked(d["A"], d["sa"], d["ld_sa"], d["B"], d["sb"], d["masked_m"], G, Mmax, N, K)
+    mm = np.minimum(d["masked_m"], Mmax)
+    live = np.arange(Mmax)[None, :] < mm[:, None]
+    for v in variants(g, "masked_"):
+        got = masked_gpu(g, d, v)
+        name = g.variant_names()[v]
+        assert np.all(got[~live] == CANARY), f"{name}: masked row written"
+        if exact:
+            assert np.array_equal(got[live], bf[live]), name
+        else:
+            assert_close(got[live], ex[live], name)
+
+
+@pytest.mark.parametrize("Mmax,mm", [(40, [0, 1, 39, 40]), (130, [129, 64, 0, 1, 130, 65]),
+                                     (256, [255, 256, 0, 1, 127, 128, 129])])
+def test_masked_edge_counts(g, Mmax, mm):
+    d = synth.masked_inputs(30 + Mmax, len(mm), Mmax, 136, 256, masked_m=mm)
+    check_masked(g, d)
+    assert g.device_error() == 0
+
+
+def test_masked_exact_integers(g):
+    G, Mmax, N, K = 3, 160, 264, 384
+    d = synth.masked_inputs(31, G, Mmax, N, K, masked_m=[160, 33, 97])
+    rng = np.random.default_rng(6)
+    d["A"] = exact_integer_codes(rng, d["A"].shape)
+    d["B"] = exact_integer_codes(rng, d["B"].shape)
+    d["sa"][:, :, :Mmax] = pow2_scales(rng, (G, K // 128, Mmax))
+    d["sb"] = pow2_scales(rng, d["sb"].shape)
+    check_masked(g, d, exact=True)
+
+
+def test_masked_count_above_mmax_is_clamped_and_flagged(g):
+    d = synth.masked_inputs(32, 2, 64, 64, 128, masked_m=[64, 64])
+    ref = masked_gpu(g, d)
+    d["masked_m"] = np.array([1000, 64], np.int32)
+    g.device_error(clear=True)
+    got = masked_gpu(g, d)
+    assert np.array_equal(got, ref)
+    assert g.device_error() & g.DEVERR_MASKED_OVER
+
+
+def test_masked_expected_m_does_not_change_results(g):
+    d = synth.masked_inputs(33, 4, 128, 264, 256, masked_m=[5, 128, 70, 0])
+    a = masked_gpu(g, d, expected_m=1)
+    b = masked_gpu(g, d, expected_m=128)
+    assert np.array_equal(a, b)
+
+
+def test_masked_in_cuda_graph_reads_counts_on_device(g):
+    """The host never reads masked_m: a captured graph replays with new counts."""
+    d = synth.masked_inputs(34, 4, 128, 136, 256, masked_m=[128, 128, 128, 128])
+    A, sa, B, sb = dev(d["A"]), dev(d["sa"]), dev(d["B"]), dev(d["sb"])
+    mm = dev(np.array([128, 128, 128, 128], np.int32))
+    D = canary_like((4, 128, 136))
+    g.m_grouped_fp8_gemm_nt_masked(A, sa, B, sb, mm, 64, D=D)  # warm-up (per-device set-up)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        g.m_grouped_fp8_gemm_nt_masked(A, sa, B, sb, mm, 64, D=D)
+    new = np.array([3, 0, 100, 128], np.int32)
+    mm.copy_(torch.from_numpy(new))
+    D.view(torch.int16).fill_(CANARY - 0x10000)
+    graph.replay()
+    got = host_bits(D)
+    d["masked_m"] = new
+    ex, _ = oracle.m_grouped_masked(d["A"], d["sa"], d["ld_sa"], d["B"], d["sb"], new, 4, 128, 136, 256)
+    live = np.arange(128)[None, :] < new[:, None]
+    assert np.all(got[~live] == CANARY)
+    assert_close(got[live], ex[live], "graph replay")
+
+
+# --------------------------------------------------------------------------- full-size configurations
+
+@pytest.mark.slow
+def test_config_dense_4096x7168x16384_sampled_rows(g):
+    d = synth.config_inputs("dense_4096x7168x16384")
+    got = dense_gpu(g, d)
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.r_[0, 4095, 127, 128, rng.choice(4096, 44, replace=False)]).astype(np.int32)
+    ex, _ = oracle_dense(d, rows=rows)
+    assert_close(got[rows], ex, "dense_4096x7168x16384 sampled")
+
+
+@pytest.mark.slow
+def test_config_contiguous_sampled_rows(g):
+    d = synth.config_inputs("contiguous_g4_m8192_n4096_k7168")
+    D = canary_like((d["M"], d["N"]))
+    g.m_grouped_fp8_gemm_nt_contiguous(dev(d["A"]), dev(d["sa"]), dev(d["B"]), dev(d["sb"]),
+                                       dev(d["m_indices"]), D=D)
+    got = host_bits(D)
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.r_[[8192 * e + o for e in range(4) for o in (0, 8191)],
+                           rng.choice(d["M"], 56, replace=False)]).astype(np.int32)
+    ex, _ = oracle.m_grouped_contiguous(d["A"], d["sa"], d["ld_sa"], d["B"], d["sb"], d["m_indices"], d["M"],
+                                        d["N"], d["K"], d["G"], rows=rows)
+    assert_close(got[rows], ex, "contiguous sampled")
+
+
+@pytest.mark.slow
+def test_config_masked_sampled_rows(g):
+    d = synth.config_inputs("masked_g16_m256_n4096_k7168")
+    got = masked_gpu(g, d, expected_m=d["expected_m"])
+    G, Mmax, N, K = d["G"], d["Mmax"], d["N"], d["K"]
+    mm = d["masked_m"]
+    live = np.arange(Mmax)[None, :] < mm[:, None]
+    assert np.all(got[~live] == CANARY)
+    rng = np.random.default_rng(2)
+    for gi in range(G):
+        if mm[gi] == 0:
+            continue
+        rows = np.unique(np.r_[0, mm[gi] - 1, rng.choice(mm[gi], min(6, mm[gi]), replace=False)]).astype(np.int32)
+        # one group's masked rows are that group's dense product (pinned in the oracle tests)
+        ex, _ = oracle.gemm_nt(d["A"][gi], d["sa"][gi], d["ld_sa"], d["B"][gi], d["sb"][gi], Mmax, N, K,
+                               rows=rows)
+        assert_close(got[gi][rows], ex, f"masked group {gi}")
