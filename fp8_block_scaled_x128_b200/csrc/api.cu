@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -25,19 +26,21 @@ struct Variant {
   int kind;
   bool swap;
   int bnc, stages, split;
+  bool reg_split;  // setmaxnreg variant: needs exactly kLaunchRegs at launch
   KernelFn fn;
   int smem;
 };
 
 template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT>
 Variant make_variant(const char* name) {
-  return Variant{name, KIND, kSwap, BNC, STAGES, SPLIT,
-                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT>,
-                 Layout<kSwap, BNC, STAGES, SPLIT>::kSmemAlloc};
+  using L = Layout<kSwap, BNC, STAGES, SPLIT>;
+  return Variant{name, KIND, kSwap, BNC, STAGES, SPLIT, L::kRegSplit,
+                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT>, L::kSmemAlloc};
 }
 
+// "nlanes": TMEM lanes are rows of B (small M); "mlanes": lanes are rows of A.
 const Variant kVariants[] = {
-    make_variant<true, 64, 7, kDense, 8>("dense_nlanes_bn64_st7_splitk8"),
+    make_variant<true, 64, 6, kDense, 8>("dense_nlanes_bn64_st6_splitk8"),
     make_variant<true, 64, 8, kDense, 1>("dense_nlanes_bn64_st8"),
     make_variant<true, 128, 6, kDense, 1>("dense_nlanes_bn128_st6"),
     make_variant<false, 128, 6, kDense, 1>("dense_mlanes_bn128_st6"),
@@ -46,6 +49,11 @@ const Variant kVariants[] = {
     make_variant<true, 64, 8, kMasked, 1>("masked_nlanes_bn64_st8"),
     make_variant<true, 128, 6, kMasked, 1>("masked_nlanes_bn128_st6"),
     make_variant<false, 128, 6, kMasked, 1>("masked_mlanes_bn128_st6"),
+    make_variant<true, 64, 6, kDense, 4>("dense_nlanes_bn64_st6_splitk4"),
+    make_variant<true, 64, 6, kDense, 2>("dense_nlanes_bn64_st6_splitk2"),
+    make_variant<false, 256, 4, kDense, 1>("dense_mlanes_bn256_st4"),
+    make_variant<false, 256, 4, kContiguous, 1>("contiguous_mlanes_bn256_st4"),
+    make_variant<false, 256, 4, kMasked, 1>("masked_mlanes_bn256_st4"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
@@ -58,9 +66,24 @@ enum : int {
   V_MASKED_N64 = 6,
   V_MASKED_N128 = 7,
   V_MASKED_M128 = 8,
+  V_DENSE_SPLIT4 = 9,
+  V_DENSE_SPLIT2 = 10,
+  V_DENSE_M256 = 11,
+  V_CONTIG_M256 = 12,
+  V_MASKED_M256 = 13,
 };
 
 std::atomic<int> g_override{-1};
+
+// Programmatic dependent launch is on unless FP8G_DISABLE_PDL is set to a
+// nonzero value in the environment (read once).
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("FP8G_DISABLE_PDL");
+    return !(e && *e && std::strcmp(e, "0") != 0);
+  }();
+  return on;
+}
 thread_local int t_last_variant = -1;
 
 // ---------------------------------------------------------------- devices
@@ -104,6 +127,13 @@ int prepare_variant(DeviceInfo* d, int v) {
   if (d->attr_set[v]) return FP8G_OK;
   const Variant& V = kVariants[v];
   if (V.smem > d->max_smem_optin) return FP8G_ERR_UNSUPPORTED;
+  if (V.reg_split) {
+    // the setmaxnreg split is sized for exactly kLaunchRegs per thread at
+    // launch; any other count would leave the promotion warps waiting
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(V.fn)) != cudaSuccess) return FP8G_ERR_CUDA;
+    if (fa.numRegs != kLaunchRegs) return FP8G_ERR_UNSUPPORTED;
+  }
   if (cudaFuncSetAttribute(reinterpret_cast<const void*>(V.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
                            V.smem) != cudaSuccess)
     return FP8G_ERR_CUDA;
@@ -241,21 +271,30 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   if (rc) return rc;
 
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  unsigned nattr = 0;
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = V.smem;
   cfg.stream = stream;
+  if (pdl_enabled()) {
+    // the kernel may start its prologue while the previous kernel in the
+    // stream finishes; it waits for that kernel before touching memory
+    attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[nattr].val.programmaticStreamSerializationAllowed = 1;
+    ++nattr;
+  }
   if (V.split > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = V.split;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[nattr].id = cudaLaunchAttributeClusterDimension;
+    attr[nattr].val.clusterDim.x = V.split;
+    attr[nattr].val.clusterDim.y = 1;
+    attr[nattr].val.clusterDim.z = 1;
+    ++nattr;
     cfg.gridDim = dim3(p.num_tiles * V.split, 1, 1);
   } else {
     cfg.gridDim = dim3(std::min(p.num_tiles, dev->sms), 1, 1);
   }
+  cfg.attrs = attr;
+  cfg.numAttrs = nattr;
   void* args[] = {&tmA, &tmB, &tmSA, &p};
   if (cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(V.fn), args) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -268,16 +307,28 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
 int select_variant(const Problem& P, DeviceInfo* dev) {
   const int ov = g_override.load(std::memory_order_relaxed);
   if (ov >= 0) return ov;
-  if (P.kind == kContiguous) return V_CONTIG_M128;
+  // m-lanes, 256 columns when there are enough such tiles to fill the GPU
+  auto wide = [&](int v256, int v128, long tiles256) {
+    return tiles256 >= dev->sms && prepare_variant(dev, v256) == FP8G_OK ? v256 : v128;
+  };
+  if (P.kind == kContiguous)
+    return wide(V_CONTIG_M256, V_CONTIG_M128, static_cast<long>(P.M / 128) * ((P.N + 255) / 256));
   if (P.kind == kMasked) return P.expected_m > 0 && P.expected_m <= 64 ? V_MASKED_N64 : V_MASKED_N128;
   if (P.M <= 64) {
+    // decode shapes: few 128-row tiles of B.  Split K over a cluster so that
+    // many SMs stream B; take the largest split whose clusters are all
+    // co-resident and that leaves each CTA at least 4 K-blocks.
     const int nt = (P.N + 127) / 128;
-    if (P.K / 128 >= 16 && prepare_variant(dev, V_DENSE_SPLIT) == FP8G_OK &&
-        nt <= dev->max_clusters[V_DENSE_SPLIT] && nt * 8 <= dev->sms)
-      return V_DENSE_SPLIT;
+    const int kb = P.K / 128;
+    for (int v : {V_DENSE_SPLIT, V_DENSE_SPLIT4, V_DENSE_SPLIT2}) {
+      const int split = kVariants[v].split;
+      if (kb < 4 * split || nt * split > dev->sms) continue;
+      if (prepare_variant(dev, v) != FP8G_OK) continue;
+      if (nt <= dev->max_clusters[v]) return v;
+    }
     return V_DENSE_N64;
   }
-  return V_DENSE_M128;
+  return wide(V_DENSE_M256, V_DENSE_M128, static_cast<long>((P.M + 127) / 128) * ((P.N + 255) / 256));
 }
 
 int run(const Problem& P, cudaStream_t stream) {

@@ -9,21 +9,28 @@
 // own design is a Hopper one (wgmma, register accumulators); this is a
 // Blackwell design:
 //
-//   warp 0        TMA producer: for every (tile, K-block) fills one stage of a
-//                 shared-memory ring with the 128-row "lane" operand tile,
-//                 the "column" operand tile and the tile's slice of sa.
-//   warp 1        MMA issuer (one thread): four tcgen05.mma kind::f8f6f4
-//                 (K = 32 each) write the K-block partial P_kb, FP32, into one
-//                 of several tensor-memory (TMEM) buffers; tcgen05.commit
-//                 frees the smem stage and signals the partial.
-//   warp 2        scale warp: turns the stage's sa slice and the tile's sb
-//                 row into the factors the promotion needs.
-//   warp 3        idle (completes warpgroup 0).
+//   warps 0, 3    TMA producers: for every (tile, K-block) one stage of a
+//                 shared-memory ring receives the 128-row "lane" operand
+//                 tile, the "column" operand tile and the tile's slice of sa.
+//                 Lanes 0..3 of both warps issue; stage s belongs to issuer
+//                 s % 8 for every round (one thread issues only about one
+//                 TMA operation per 150 ns, which would cap a CTA near
+//                 50 GB/s).
+//   warps 1, 2    MMA issuers (lane 0 of each; stage s belongs to issuer
+//                 s % 2): four tcgen05.mma kind::f8f6f4 (K = 32 each) write
+//                 the K-block partial P_kb, FP32, into one of several
+//                 tensor-memory (TMEM) buffers; tcgen05.commit frees the
+//                 stage and signals the partial.  A single thread spends
+//                 about 650 cycles per K-block on waits, MMA issue and
+//                 commits, more than an N <= 128 MMA takes to execute; two
+//                 issuers overlap that work.
 //   warps 4..11   two promotion warpgroups, each owning half the tile's
 //                 columns: tcgen05.ld the finished partial, acc += P * scale
 //                 in FP32 registers (CUDA cores), release the TMEM buffer so
 //                 the MMA of a later K-block overlaps; after the tile's last
-//                 K-block, round to bf16 and store D.
+//                 K-block, round to bf16 and store D.  The sb values of the
+//                 tile are prefetched 32 K-blocks at a time into a register
+//                 per lane and broadcast with a shuffle.
 //
 // Orientation.  The MMA's M side (TMEM lanes) is always 128 rows.
 //   kSwap = true : lanes are 128 rows of B (n), columns are BNC rows of A
@@ -32,12 +39,20 @@
 //                  (tile, K-block) and the A scale varies per column.
 //   kSwap = false: lanes are 128 rows of A (m), columns are BNC rows of B.
 //                  The A scale is one scalar per thread, the B scale one per
-//                  128 columns.
+//                  128 columns.  With BNC = 256 each promotion thread holds
+//                  128 accumulators, so the warpgroups trade registers with
+//                  setmaxnreg (control 56, promotion 224 per thread).
 // Scheduling kinds: dense; contiguous (128-row blocks of A map to experts via
 // m_indices, -1 = skip); masked (tiles at or past masked_m[g] are skipped).
 // SPLIT > 1 (dense, kSwap only): a cluster of SPLIT CTAs shares one output
-// tile, each over K/SPLIT, and the partial sums are reduced through
-// distributed shared memory in a fixed order (deterministic).
+// tile, each over K/SPLIT.  Each CTA stores its partial sums into the shared
+// memory of the CTA that owns those columns; after one cluster barrier every
+// CTA adds the SPLIT partials of its columns in rank order (deterministic).
+//
+// Programmatic dependent launch: the prologue (barrier init, TMEM
+// allocation, tensor-map prefetch) runs before griddepcontrol.wait, so it can
+// overlap the previous kernel in the stream; no global memory is touched
+// before that wait.
 //
 // Every wait is bounded: after kWaitTimeoutNs the waiter records
 // FP8G_DEVERR_TIMEOUT, raises a CTA-wide abort flag, and every role leaves
@@ -60,6 +75,8 @@ namespace fp8g {
 enum Kind : int { kDense = 0, kContiguous = 1, kMasked = 2 };
 
 constexpr int kThreads = 384;
+constexpr int kIssuersPerWarp = 4;                  // TMA-issuing lanes in each producer warp
+constexpr int kIssuers = 2 * kIssuersPerWarp;       // warps 0 and 3
 constexpr int kKBMax = 512;                         // K <= 65536
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s
 constexpr uint64_t kDrainTimeoutNs = 100000000ull;  // 0.1 s
@@ -90,20 +107,18 @@ struct Layout {
   static constexpr int kLaneBytes = 128 * 128;   // 128 rows x 128 e4m3 (one K-block)
   static constexpr int kColBytes = BNC * 128;
   static constexpr int kSaFloats = kSwap ? BNC : 128;  // sa slice: the tile's m-extent
-  static constexpr int kSclFloats = kSwap ? BNC : 4;   // scale factors per stage
   static constexpr int kNBuf = BNC <= 128 ? 4 : 2;     // TMEM partial buffers
   static constexpr int kTmemCols = pow2_at_least(kNBuf * BNC, 32);
   static constexpr int kCW = BNC / 2;                  // columns per promotion warpgroup
+  static constexpr bool kRegSplit = kCW > 64;          // 128 accumulators per thread
   static constexpr int kCPD = BNC / SPLIT;             // split-K: columns reduced per CTA
   static constexpr int kOffLane = 0;
   static constexpr int kOffCol = kOffLane + STAGES * kLaneBytes;
   static constexpr int kOffSa = kOffCol + STAGES * kColBytes;
-  static constexpr int kOffScl = kOffSa + STAGES * kSaFloats * 4;
-  static constexpr int kOffSbRow = kOffScl + STAGES * kSclFloats * 4;
-  static constexpr int kOffRecv = kOffSbRow + 2 * kKBMax * 4;
+  static constexpr int kOffRecv = kOffSa + STAGES * kSaFloats * 4;
   static constexpr int kRecvBytes = SPLIT > 1 ? SPLIT * 128 * kCPD * 4 : 0;
   static constexpr int kOffBar = kOffRecv + kRecvBytes;
-  static constexpr int kNumBars = 3 * STAGES + 2 * kNBuf + 2;
+  static constexpr int kNumBars = 2 * STAGES + 2 * kNBuf + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;  // + slack to align the base to 1024
@@ -111,12 +126,21 @@ struct Layout {
   static_assert(BNC % 32 == 0 && BNC >= 32 && BNC <= 256, "column tile");
   static_assert(kCW % 32 == 0, "promotion chunking");
   static_assert(kTmemCols <= 512, "TMEM");
+  static_assert(STAGES % 2 == 0 && kNBuf % 2 == 0, "stages and TMEM buffers alternate between the two MMA issuers");
   static_assert(kOffCol % 1024 == 0 && kOffSa % 1024 == 0, "swizzle-128B tiles need 1024 alignment");
   static_assert(kColBytes % 1024 == 0, "column tile rows must be a multiple of 8");
   static_assert(SPLIT == 1 || (kSwap && BNC % SPLIT == 0 && kCW % kCPD == 0 && kCPD % 4 == 0),
                 "split-K layout");
+  static_assert(!kRegSplit || !kSwap, "the register split is for the m-lanes orientation");
   static_assert(kSmemAlloc <= 232448, "shared memory");
 };
+
+// Register budget of the BNC = 256 variants: 384 threads launch with 168
+// registers each (the compiler's cap for 384 threads per SM); the control
+// warpgroup gives back 112 per thread and the two promotion warpgroups take
+// 56 more each: 128 * (168 - 56) == 256 * (224 - 168).
+constexpr int kLaunchRegs = 168, kControlRegs = 56, kPromoRegs = 224;
+static_assert(128 * (kLaunchRegs - kControlRegs) == 256 * (kPromoRegs - kLaunchRegs), "register split");
 
 struct Tile {
   int g, m0, n0, mvalid, kb0, kb1;
@@ -221,11 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar0 = sbase + L::kOffBar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto scl_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
-  auto tfull_bar = [&](int b) { return bar0 + 8u * (3 * STAGES + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (3 * STAGES + L::kNBuf + b); };
-  const uint32_t recv_bar = bar0 + 8u * (3 * STAGES + 2 * L::kNBuf);
-  const uint32_t drain_bar = recv_bar + 8u;
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + L::kNBuf + b); };
+  auto drain_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + 2 * L::kNBuf + i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -233,23 +255,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto lane_tile = [&](int s) { return sbase + L::kOffLane + s * L::kLaneBytes; };
   auto col_tile = [&](int s) { return sbase + L::kOffCol + s * L::kColBytes; };
   auto sa_slice = [&](int s) { return sbase + L::kOffSa + s * L::kSaFloats * 4; };
-  float* sa_f = reinterpret_cast<float*>(smem + L::kOffSa);
-  float* scl_f = reinterpret_cast<float*>(smem + L::kOffScl);
-  float* sbrow = reinterpret_cast<float*>(smem + L::kOffSbRow);
+  const float* sa_f = reinterpret_cast<const float*>(smem + L::kOffSa);
 
   constexpr int kPromoWarps = 8;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1 + kPromoWarps);
-      mbar_init(scl_bar(s), 1);
+      mbar_init(empty_bar(s), 1 + kPromoWarps);  // MMA commit + promotion warps (they read sa)
     }
     for (int b = 0; b < L::kNBuf; ++b) {
       mbar_init(tfull_bar(b), 1);
       mbar_init(tempty_bar(b), kPromoWarps);
     }
-    mbar_init(recv_bar, SPLIT * 128);
-    mbar_init(drain_bar, 1);
+    mbar_init(drain_bar(0), 1);
+    mbar_init(drain_bar(1), 1);
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -267,15 +286,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if constexpr (SPLIT > 1) cluster_sync_all();
   const uint32_t tmem_base = *tmem_slot;
+  // inputs may be written by the previous kernel in the stream: wait for it
+  // (a no-op without a programmatic dependency), then let the next one start
+  // its own prologue
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
 
   const uint32_t rank = SPLIT > 1 ? cluster_ctarank() : 0u;
   const int t_first = SPLIT > 1 ? static_cast<int>(blockIdx.x) / SPLIT : static_cast<int>(blockIdx.x);
   const int t_step = SPLIT > 1 ? p.num_tiles : static_cast<int>(gridDim.x);
   constexpr uint32_t kStageTx = L::kLaneBytes + L::kColBytes + L::kSaFloats * 4;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp < 4) {
+  if constexpr (L::kRegSplit) setmaxnreg_dec<kControlRegs>();
+  if (warp == 0 || warp == 3) {
+    // ------------------------------------------------------------ producers
+    if (lane < kIssuersPerWarp) {
+      const uint32_t me = static_cast<uint32_t>((warp == 3 ? kIssuersPerWarp : 0) + lane);
       uint32_t it = 0;
       bool ok = true;
       for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
@@ -284,6 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ga = KIND == kMasked ? T.g : 0;
         const int gb = KIND == kDense ? 0 : T.g;
         for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
+          // a stage always has the same issuer, which walks its rounds in
+          // order; the parity wait below is only unambiguous under that rule
+          if ((it % STAGES) % kIssuers != me) continue;
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag)) {
@@ -301,24 +331,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(sa_slice(s), &tmSA, full_bar(s), T.m0, kb, ga);
         }
       }
-      // drain: every issued load must land before the CTA may exit
+      // drain: every load this thread issued must land before the CTA exits
+      // (the last STAGES iterations use distinct stages)
       const uint32_t first = it > static_cast<uint32_t>(STAGES) ? it - STAGES : 0u;
-      for (uint32_t i = first; i < it; ++i) drain_phase(full_bar(i % STAGES), (i / STAGES) & 1u);
+      for (uint32_t i = first; i < it; ++i)
+        if ((i % STAGES) % kIssuers == me) drain_phase(full_bar(i % STAGES), (i / STAGES) & 1u);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
+      const uint32_t me = static_cast<uint32_t>(warp - 1);
       constexpr uint32_t kIdesc = idesc_e4m3_f32(128, BNC);
-      uint32_t it = 0, tb = 0;
+      uint32_t it = 0;
       bool ok = true;
       for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
         const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t, rank, false);
         if (!T.valid) continue;
-        for (int kb = T.kb0; kb < T.kb1; ++kb, ++it, ++tb) {
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
+          // stage s and TMEM buffer it % kNBuf (both even counts) belong to
+          // issuer s % 2 in every round
+          if ((it % STAGES) % 2 != me) continue;
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          const int b = tb % L::kNBuf;
-          const uint32_t tph = (tb / L::kNBuf) & 1u;
+          const int b = it % L::kNBuf;
+          const uint32_t tph = (it / L::kNBuf) & 1u;
           if (!wait_phase(full_bar(s), ph, abort_flag) ||
               !wait_phase(tempty_bar(b), tph ^ 1u, abort_flag)) {
             ok = false;
@@ -337,69 +373,49 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(tfull_bar(b));
         }
       }
-      // drain: all issued MMAs complete before TMEM is freed
-      mma_commit(drain_bar);
-      drain_phase(drain_bar, 0u);
+      // drain: all MMAs this thread issued complete before TMEM is freed
+      mma_commit(drain_bar(me));
+      drain_phase(drain_bar(me), 0u);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ scale warp
-    uint32_t it = 0;
-    bool ok = true;
-    for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
-      const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t, rank, lane == 0);
-      if (!T.valid) continue;
-      // this tile's sb rows for its K-block range
-      constexpr int kRows = kSwap ? 1 : BNC / 128;
-      const int nkb = T.kb1 - T.kb0;
-      for (int j = 0; j < kRows; ++j) {
-        const int nb = T.n0 / 128 + j;
-        const float* src = p.sb + (static_cast<long>(T.g) * p.NB + nb) * p.KB + T.kb0;
-        for (int i = lane; i < nkb; i += 32) sbrow[j * kKBMax + i] = nb < p.NB ? __ldg(src + i) : 0.f;
-      }
-      __syncwarp();
-      for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1u;
-        const bool w = wait_phase(full_bar(s), ph, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
-        if constexpr (kSwap) {
-          const float sbv = sbrow[kb - T.kb0];
-          const float* sa_s = sa_f + s * L::kSaFloats;
-          float* out = scl_f + s * L::kSclFloats;
-          for (int c = lane; c < BNC; c += 32) out[c] = sa_s[c] * sbv;
-        } else {
-          if (lane < kRows) scl_f[s * L::kSclFloats + lane] = sbrow[lane * kKBMax + (kb - T.kb0)];
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(scl_bar(s));
-      }
-    }
-  } else if (warp >= 4) {
+  }
+  } else {
     // ------------------------------------------------------------ promotion + epilogue
+    if constexpr (L::kRegSplit) setmaxnreg_inc<kPromoRegs>();
     constexpr int kCW = L::kCW;
     const int wg = (warp - 4) / 4;  // column half
     const int q = warp % 4;         // TMEM lane quarter this warp may access
     const int row = 32 * q + lane;  // tile row = TMEM lane
     float acc[kCW];
-    uint32_t it = 0, tb = 0;
+    uint32_t it = 0;
     bool ok = true;
     for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
-      const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t, rank, false);
+      // one thread records bad m_indices / masked_m entries in the error word
+      const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t, rank, warp == 4 && lane == 0);
       if (!T.valid) continue;
 #pragma unroll
       for (int c = 0; c < kCW; ++c) acc[c] = 0.f;
       // column chunks of 32 that hold valid output (kSwap: columns are rows of A)
       const int live = kSwap ? min(kCW, max(0, T.mvalid - wg * kCW)) : kCW;
-      for (int kb = T.kb0; kb < T.kb1; ++kb, ++it, ++tb) {
+      // the sb row of this thread's columns, 32 K-blocks per register (lane i
+      // holds K-block kb0 + 32j + i), the next chunk loaded one chunk ahead
+      const int nb = min((kSwap ? T.n0 : T.n0 + wg * kCW) / 128, p.NB - 1);
+      const float* sbp = p.sb + (static_cast<long>(T.g) * p.NB + nb) * p.KB;
+      float sb_cur = T.kb0 + lane < T.kb1 ? __ldg(sbp + T.kb0 + lane) : 0.f;
+      float sb_nxt = T.kb0 + 32 + lane < T.kb1 ? __ldg(sbp + T.kb0 + 32 + lane) : 0.f;
+      for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
-        const int b = tb % L::kNBuf;
-        const uint32_t tph = (tb / L::kNBuf) & 1u;
+        const int b = it % L::kNBuf;
+        const uint32_t tph = (it / L::kNBuf) & 1u;
+        const int i32 = (kb - T.kb0) & 31;
+        if (i32 == 0 && kb != T.kb0) {
+          sb_cur = sb_nxt;
+          sb_nxt = kb + 32 + lane < T.kb1 ? __ldg(sbp + kb + 32 + lane) : 0.f;
+        }
+        const float s_b = __shfl_sync(0xffffffffu, sb_cur, i32);
+        // the stage's sa slice is read below: wait for its TMA as well
         bool w = wait_phase(tfull_bar(b), tph, abort_flag);
-        w = w && wait_phase(scl_bar(s), ph, abort_flag);
+        w = w && wait_phase(full_bar(s), ph, abort_flag);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
@@ -407,35 +423,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
                                static_cast<uint32_t>(b * BNC + wg * kCW);
-        uint32_t r[kCW / 32][32];
+        // this thread's scale: sa[m0 + row, kb] * sb[nb, kb] (m-lanes), or
+        // per column sa[m0 + c, kb] * sb[nb, kb] (n-lanes)
+        const float sc_row = kSwap ? 0.f : sa_f[s * L::kSaFloats + row] * s_b;
+        // chunks of 32 columns, loaded two at a time (64 staging registers)
+        constexpr int kChunks = kCW / 32;
+        constexpr int kGroup = kChunks < 2 ? kChunks : 2;
 #pragma unroll
-        for (int j = 0; j < kCW / 32; ++j)
-          if (32 * j < live) tmem_ld_32x32b_x32(taddr + 32 * j, r[j]);
-        tmem_ld_wait_bind(r[0]);
+        for (int j0 = 0; j0 < kChunks; j0 += kGroup) {
+          if (32 * j0 >= live) break;
+          uint32_t r[kGroup][32];
 #pragma unroll
-        for (int j = 1; j < kCW / 32; ++j) bind_after_wait(r[j]);
-        if constexpr (kSwap) {
-          const float4* f4 = reinterpret_cast<const float4*>(scl_f + s * L::kSclFloats + wg * kCW);
+          for (int j = 0; j < kGroup; ++j)
+            if (32 * (j0 + j) < live) tmem_ld_32x32b_x32(taddr + 32 * (j0 + j), r[j]);
+          tmem_ld_wait_bind(r[0]);
 #pragma unroll
-          for (int j = 0; j < kCW / 32; ++j) {
-            if (32 * j < live) {
+          for (int j = 1; j < kGroup; ++j) bind_after_wait(r[j]);
+#pragma unroll
+          for (int j = 0; j < kGroup; ++j) {
+            if (32 * (j0 + j) >= live) continue;
+            float* a = acc + 32 * (j0 + j);
+            if constexpr (kSwap) {
+              const float4* f4 = reinterpret_cast<const float4*>(sa_f + s * L::kSaFloats + wg * kCW + 32 * (j0 + j));
 #pragma unroll
               for (int c4 = 0; c4 < 8; ++c4) {
-                const float4 f = f4[8 * j + c4];
-                float* a = acc + 32 * j + 4 * c4;
-                a[0] = fmaf(__uint_as_float(r[j][4 * c4 + 0]), f.x, a[0]);
-                a[1] = fmaf(__uint_as_float(r[j][4 * c4 + 1]), f.y, a[1]);
-                a[2] = fmaf(__uint_as_float(r[j][4 * c4 + 2]), f.z, a[2]);
-                a[3] = fmaf(__uint_as_float(r[j][4 * c4 + 3]), f.w, a[3]);
+                const float4 f = f4[c4];
+                a[4 * c4 + 0] = fmaf(__uint_as_float(r[j][4 * c4 + 0]), f.x * s_b, a[4 * c4 + 0]);
+                a[4 * c4 + 1] = fmaf(__uint_as_float(r[j][4 * c4 + 1]), f.y * s_b, a[4 * c4 + 1]);
+                a[4 * c4 + 2] = fmaf(__uint_as_float(r[j][4 * c4 + 2]), f.z * s_b, a[4 * c4 + 2]);
+                a[4 * c4 + 3] = fmaf(__uint_as_float(r[j][4 * c4 + 3]), f.w * s_b, a[4 * c4 + 3]);
               }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc_row, a[c]);
             }
           }
-        } else {
-          const float sc = sa_f[s * L::kSaFloats + row] * scl_f[s * L::kSclFloats + (wg * kCW) / 128];
-#pragma unroll
-          for (int j = 0; j < kCW / 32; ++j)
-#pragma unroll
-            for (int c = 0; c < 32; ++c) acc[32 * j + c] = fmaf(__uint_as_float(r[j][c]), sc, acc[32 * j + c]);
         }
         tc_fence_before();
         __syncwarp();
@@ -448,7 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       const long drow0 = KIND == kMasked ? static_cast<long>(T.g) * p.M : 0;
       if constexpr (SPLIT > 1) {
-        // push this CTA's partial columns to the CTA that reduces them
+        // store this CTA's partial columns into the shared memory of the CTA
+        // that reduces them (slot = this CTA's rank); the reduction follows
+        // the cluster barrier after the role loops
         constexpr int kCPD = L::kCPD;
         const uint32_t recv_local = sbase + L::kOffRecv + (rank * 128u + row) * (kCPD * 4u);
 #pragma unroll
@@ -458,39 +482,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < kCPD; c += 4)
             st_cluster_v4(raddr + 4u * c, acc[d0 + c], acc[d0 + c + 1], acc[d0 + c + 2], acc[d0 + c + 3]);
-          mbar_arrive_remote(mapa(recv_bar, dst));
-        }
-        // reduce the columns this CTA owns, in source-rank order
-        if (wg == static_cast<int>((rank * kCPD) / kCW)) {
-          const bool w = wait_phase<true>(recv_bar, 0u, abort_flag);
-          if (!__all_sync(0xffffffffu, w)) {
-            ok = false;
-            break;
-          }
-          float sum[kCPD];
-#pragma unroll
-          for (int c = 0; c < kCPD; ++c) sum[c] = 0.f;
-          const float* rv = reinterpret_cast<const float*>(smem + L::kOffRecv);
-          for (int src = 0; src < SPLIT; ++src) {
-            const float4* v = reinterpret_cast<const float4*>(rv + (src * 128 + row) * kCPD);
-#pragma unroll
-            for (int c4 = 0; c4 < kCPD / 4; ++c4) {
-              const float4 f = v[c4];
-              sum[4 * c4 + 0] += f.x;
-              sum[4 * c4 + 1] += f.y;
-              sum[4 * c4 + 2] += f.z;
-              sum[4 * c4 + 3] += f.w;
-            }
-          }
-          const int n = T.n0 + row;
-          if (n < p.N) {
-#pragma unroll
-            for (int c = 0; c < kCPD; ++c) {
-              const int mc = static_cast<int>(rank) * kCPD + c;
-              if (mc < T.mvalid)
-                p.D[(drow0 + T.m0 + mc) * p.N + n] = static_cast<uint16_t>(pack_bf16x2(sum[c], 0.f) & 0xFFFFu);
-            }
-          }
         }
       } else if constexpr (kSwap) {
         // lanes hold consecutive n: each column store is 64 contiguous bytes per warp
@@ -521,15 +512,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // ------------------------------------------------------------ teardown
   __syncwarp();
+  if constexpr (SPLIT > 1) {
+    // all partials of this cluster's tile are in place after the barrier;
+    // the warpgroup whose columns this CTA owns adds them in rank order
+    cluster_sync_all();
+    constexpr int kCPD = L::kCPD;
+    const int wg = (warp - 4) / 4;
+    if (warp >= 4 && !*abort_flag && wg == static_cast<int>((rank * kCPD) / L::kCW)) {
+      const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t_first, rank, false);
+      const int row = 32 * (warp % 4) + lane;
+      float sum[kCPD];
+#pragma unroll
+      for (int c = 0; c < kCPD; ++c) sum[c] = 0.f;
+      const float* rv = reinterpret_cast<const float*>(smem + L::kOffRecv);
+      for (int src = 0; src < SPLIT; ++src) {
+        const float4* v = reinterpret_cast<const float4*>(rv + (src * 128 + row) * kCPD);
+#pragma unroll
+        for (int c4 = 0; c4 < kCPD / 4; ++c4) {
+          const float4 f = v[c4];
+          sum[4 * c4 + 0] += f.x;
+          sum[4 * c4 + 1] += f.y;
+          sum[4 * c4 + 2] += f.z;
+          sum[4 * c4 + 3] += f.w;
+        }
+      }
+      const int n = T.n0 + row;
+      if (T.valid && n < p.N) {
+#pragma unroll
+        for (int c = 0; c < kCPD; ++c) {
+          const int mc = static_cast<int>(rank) * kCPD + c;
+          if (mc < T.mvalid)
+            p.D[static_cast<long>(T.m0 + mc) * p.N + n] = static_cast<uint16_t>(pack_bf16x2(sum[c], 0.f) & 0xFFFFu);
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
   }
-  if constexpr (SPLIT > 1) cluster_sync_all();  // no CTA leaves while a peer may still write to it
 }
 
 }  // namespace fp8g
