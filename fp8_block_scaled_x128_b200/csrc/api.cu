@@ -54,6 +54,7 @@ const Variant kVariants[] = {
     make_variant<false, 256, 4, kDense, 1>("dense_mlanes_bn256_st4"),
     make_variant<false, 256, 4, kContiguous, 1>("contiguous_mlanes_bn256_st4"),
     make_variant<false, 256, 4, kMasked, 1>("masked_mlanes_bn256_st4"),
+    make_variant<true, 64, 8, kDense, kGlobalSplit>("dense_nlanes_bn64_st8_gsplit"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
@@ -71,6 +72,7 @@ enum : int {
   V_DENSE_M256 = 11,
   V_CONTIG_M256 = 12,
   V_MASKED_M256 = 13,
+  V_DENSE_GSPLIT = 14,
 };
 
 std::atomic<int> g_override{-1};
@@ -96,6 +98,10 @@ struct DeviceInfo {
   int max_smem_optin = 0;
   bool attr_set[kNumVariants] = {};
   int max_clusters[kNumVariants] = {};  // split variants: co-resident clusters
+  // global split-K workspace: sms slots of 64 x 128 floats, 2 counters per tile
+  float* ws = nullptr;
+  uint32_t* sync = nullptr;
+  bool ws_failed = false;
 };
 
 std::mutex g_dev_mu;
@@ -161,6 +167,42 @@ int prepare_variant(DeviceInfo* d, int v) {
   }
   d->attr_set[v] = true;
   return FP8G_OK;
+}
+
+// The global split-K workspace of this device (sms x 64 x 128 floats and two
+// counters per tile, ~4.7 MB on B200): allocated on the first call that needs
+// it, counters zeroed.  Allocation is not allowed while `stream` is being
+// captured; the caller then uses a variant without a workspace.
+int ensure_workspace(DeviceInfo* d, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (d->ws) return FP8G_OK;
+  if (d->ws_failed) return FP8G_ERR_UNSUPPORTED;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+    (void)cudaGetLastError();
+    return FP8G_ERR_UNSUPPORTED;
+  }
+  const size_t ws_bytes = static_cast<size_t>(d->sms) * 64 * 128 * sizeof(float);
+  const size_t sync_bytes = static_cast<size_t>(d->sms) * 2 * sizeof(uint32_t);
+  void *ws = nullptr, *sync = nullptr;
+  if (cudaMalloc(&ws, ws_bytes) != cudaSuccess || cudaMalloc(&sync, sync_bytes) != cudaSuccess ||
+      cudaMemset(sync, 0, sync_bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    (void)cudaGetLastError();
+    if (ws) (void)cudaFree(ws);
+    if (sync) (void)cudaFree(sync);
+    d->ws_failed = true;
+    return FP8G_ERR_UNSUPPORTED;
+  }
+  d->ws = static_cast<float*>(ws);
+  d->sync = static_cast<uint32_t*>(sync);
+  return FP8G_OK;
+}
+
+// Split count of the global split-K variant for a decode shape: as many CTAs
+// per tile as fit one per SM, each with at least 4 K-blocks.
+int gsplit_for(const DeviceInfo* d, int tiles, int kb) {
+  if (tiles <= 0 || tiles > d->sms) return 0;
+  return std::max(1, std::min({d->sms / tiles, kb / 4, kMaxGSplit}));
 }
 
 // ---------------------------------------------------------------- tensor maps
@@ -256,6 +298,13 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   p.sb = P.sb;
   p.D = P.D;
   if (p.num_tiles <= 0) return FP8G_OK;
+  if (V.split == kGlobalSplit) {
+    p.gsplit = gsplit_for(dev, p.num_tiles, KB);
+    if (p.gsplit < 1 || p.num_tiles * p.gsplit > dev->sms) return FP8G_ERR_UNSUPPORTED;
+    if ((rc = ensure_workspace(dev, stream))) return rc;
+    p.ws = dev->ws;
+    p.sync = dev->sync;
+  }
 
   CUtensorMap tmA, tmB, tmSA;
   const uint32_t a_box_rows = V.swap ? V.bnc : 128;
@@ -290,6 +339,8 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
     attr[nattr].val.clusterDim.z = 1;
     ++nattr;
     cfg.gridDim = dim3(p.num_tiles * V.split, 1, 1);
+  } else if (V.split == kGlobalSplit) {
+    cfg.gridDim = dim3(p.num_tiles * p.gsplit, 1, 1);
   } else {
     cfg.gridDim = dim3(std::min(p.num_tiles, dev->sms), 1, 1);
   }
@@ -304,7 +355,7 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   return FP8G_OK;
 }
 
-int select_variant(const Problem& P, DeviceInfo* dev) {
+int select_variant(const Problem& P, DeviceInfo* dev, cudaStream_t stream) {
   const int ov = g_override.load(std::memory_order_relaxed);
   if (ov >= 0) return ov;
   // m-lanes, 256 columns when there are enough such tiles to fill the GPU
@@ -320,6 +371,9 @@ int select_variant(const Problem& P, DeviceInfo* dev) {
     // co-resident and that leaves each CTA at least 4 K-blocks.
     const int nt = (P.N + 127) / 128;
     const int kb = P.K / 128;
+    if (gsplit_for(dev, nt, kb) >= 2 && prepare_variant(dev, V_DENSE_GSPLIT) == FP8G_OK &&
+        ensure_workspace(dev, stream) == FP8G_OK)
+      return V_DENSE_GSPLIT;
     for (int v : {V_DENSE_SPLIT, V_DENSE_SPLIT4, V_DENSE_SPLIT2}) {
       const int split = kVariants[v].split;
       if (kb < 4 * split || nt * split > dev->sms) continue;
@@ -335,7 +389,7 @@ int run(const Problem& P, cudaStream_t stream) {
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
   if (rc) return rc;
-  const int v = select_variant(P, dev);
+  const int v = select_variant(P, dev, stream);
   if (v < 0 || v >= kNumVariants) return FP8G_ERR_UNSUPPORTED;
   return launch(P, v, dev, stream);
 }
@@ -404,6 +458,10 @@ int fp8g_get_device_error(int device, uint32_t* bits, int clear) {
     if (clear) {
       const uint32_t z = 0;
       if (cudaMemcpyToSymbol(g_fp8g_error_word, &z, sizeof(z), 0, cudaMemcpyHostToDevice) != cudaSuccess)
+        rc = FP8G_ERR_CUDA;
+      // a call that gave up can leave split-K counters behind: zero them
+      DeviceInfo* d = (device >= 0 && device < kMaxDevices) ? &g_dev[device] : nullptr;
+      if (w && d && d->sync && cudaMemset(d->sync, 0, static_cast<size_t>(d->sms) * 2 * sizeof(uint32_t)) != cudaSuccess)
         rc = FP8G_ERR_CUDA;
     }
     if (!rc && w) rc = FP8G_ERR_DEVICE;

@@ -94,7 +94,18 @@ struct Params {
   const int32_t* masked_m;
   const float* sb;  // [G][NB][KB]
   uint16_t* D;
+  // global split-K (SPLIT == kGlobalSplit): K is split over `gsplit` CTAs per
+  // tile; partials go to ws[tile][rank][BNC][128] and sync[2*tile + {0,1}]
+  // counts arrivals and departures (zero between calls: the last CTA of a
+  // tile to leave resets them)
+  int gsplit;
+  float* ws;
+  uint32_t* sync;
 };
+
+// SPLIT template value selecting the global-memory split-K (count at run time)
+constexpr int kGlobalSplit = -1;
+constexpr int kMaxGSplit = 16;  // the host never picks more
 
 constexpr int pow2_at_least(int x, int lo) {
   int p = lo;
@@ -107,11 +118,11 @@ struct Layout {
   static constexpr int kLaneBytes = 128 * 128;   // 128 rows x 128 e4m3 (one K-block)
   static constexpr int kColBytes = BNC * 128;
   static constexpr int kSaFloats = kSwap ? BNC : 128;  // sa slice: the tile's m-extent
-  static constexpr int kNBuf = BNC <= 128 ? 4 : 2;     // TMEM partial buffers
+  static constexpr int kNBuf = 512 / BNC < 8 ? 512 / BNC : 8;  // TMEM partial buffers
   static constexpr int kTmemCols = pow2_at_least(kNBuf * BNC, 32);
   static constexpr int kCW = BNC / 2;                  // columns per promotion warpgroup
   static constexpr bool kRegSplit = kCW > 64;          // 128 accumulators per thread
-  static constexpr int kCPD = BNC / SPLIT;             // split-K: columns reduced per CTA
+  static constexpr int kCPD = SPLIT > 1 ? BNC / SPLIT : BNC;  // cluster split-K: columns reduced per CTA
   static constexpr int kOffLane = 0;
   static constexpr int kOffCol = kOffLane + STAGES * kLaneBytes;
   static constexpr int kOffSa = kOffCol + STAGES * kColBytes;
@@ -129,8 +140,9 @@ struct Layout {
   static_assert(STAGES % 2 == 0 && kNBuf % 2 == 0, "stages and TMEM buffers alternate between the two MMA issuers");
   static_assert(kOffCol % 1024 == 0 && kOffSa % 1024 == 0, "swizzle-128B tiles need 1024 alignment");
   static_assert(kColBytes % 1024 == 0, "column tile rows must be a multiple of 8");
-  static_assert(SPLIT == 1 || (kSwap && BNC % SPLIT == 0 && kCW % kCPD == 0 && kCPD % 4 == 0),
-                "split-K layout");
+  static_assert(SPLIT <= 1 || (kSwap && BNC % SPLIT == 0 && kCW % kCPD == 0 && kCPD % 4 == 0),
+                "cluster split-K layout");
+  static_assert(SPLIT != kGlobalSplit || kSwap, "global split-K is for the n-lanes orientation");
   static_assert(!kRegSplit || !kSwap, "the register split is for the m-lanes orientation");
   static_assert(kSmemAlloc <= 232448, "shared memory");
 };
@@ -158,9 +170,10 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int t, uint32_t rank, 
   T.g = 0;
   T.kb0 = 0;
   T.kb1 = p.KB;
-  if constexpr (SPLIT > 1) {
-    T.kb0 = static_cast<int>((static_cast<long>(p.KB) * rank) / SPLIT);
-    T.kb1 = static_cast<int>((static_cast<long>(p.KB) * (rank + 1)) / SPLIT);
+  if constexpr (SPLIT != 1) {
+    const long ns = SPLIT > 1 ? SPLIT : p.gsplit;
+    T.kb0 = static_cast<int>((static_cast<long>(p.KB) * rank) / ns);
+    T.kb1 = static_cast<int>((static_cast<long>(p.KB) * (rank + 1)) / ns);
   }
   if constexpr (KIND == kDense) {
     const int nt = t % p.n_tiles, mt = t / p.n_tiles;
@@ -229,6 +242,69 @@ __device__ __forceinline__ void drain_phase(uint32_t bar, uint32_t parity) {
   }
 }
 
+// Global split-K reduction, run by the 256 promotion threads of every CTA of
+// a tile after they stored their partial: publish (fence + arrival count),
+// wait until all p.gsplit CTAs of the tile have published, then add the
+// partials of this CTA's columns (rows of D) in rank order and store bf16.
+// The CTAs of a tile must be resident together: the grid never exceeds the
+// SM count and the wait is bounded.
+template <int BNC, int KIND>
+__device__ __forceinline__ void global_split_reduce(const Params& p, int tile, uint32_t rank,
+                                                    volatile uint32_t* abort_flag) {
+  const int tid = threadIdx.x - 128;  // 0..255
+  uint32_t* arrive = p.sync + 2 * tile;
+  uint32_t* depart = arrive + 1;
+  named_barrier_sync(1, 256);  // every partial of this CTA is written
+  if (tid == 0) {
+    __threadfence();
+    atomicAdd(arrive, 1u);
+  }
+  // wait for the other CTAs of the tile (one poller, then the barrier)
+  if (tid == 0) {
+    const uint32_t need = static_cast<uint32_t>(p.gsplit);
+    if (ld_acquire_gpu(arrive) < need && !*abort_flag) {
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire_gpu(arrive) < need) {
+        if (*abort_flag) break;
+        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+          *abort_flag = 1u;
+          atomicOr(&g_fp8g_error_word, FP8G_DEVERR_TIMEOUT);
+          break;
+        }
+      }
+    }
+  }
+  named_barrier_sync(1, 256);
+  if (!*abort_flag) {
+    // columns [c0, c1) of the tile: rows m0 + c of D; thread -> (row, column parity)
+    const int cpd = (BNC + p.gsplit - 1) / p.gsplit;
+    const int c0 = static_cast<int>(rank) * cpd, c1 = min(BNC, c0 + cpd);
+    const int row = tid & 127;
+    const int tile_n = tile % p.n_tiles, tile_m = tile / p.n_tiles;
+    const int n = tile_n * 128 + row;
+    const int m0 = tile_m * BNC;
+    const long base = static_cast<long>(tile) * p.gsplit * (BNC * 128);
+    for (int c = c0 + (tid >> 7); c < c1; c += 2) {
+      // all partials of this element are loaded before the rank-order sum
+      float v[kMaxGSplit];
+#pragma unroll
+      for (int src = 0; src < kMaxGSplit; ++src)
+        v[src] = src < p.gsplit ? __ldcg(p.ws + base + (src * BNC + c) * 128 + row) : 0.f;
+      float sum = 0.f;
+#pragma unroll
+      for (int src = 0; src < kMaxGSplit; ++src) sum += v[src];
+      if (n < p.N && m0 + c < p.M)
+        p.D[static_cast<long>(m0 + c) * p.N + n] = static_cast<uint16_t>(pack_bf16x2(sum, 0.f) & 0xFFFFu);
+    }
+  }
+  named_barrier_sync(1, 256);  // this CTA's reads of the workspace are done
+  if (tid == 0 && atomicAdd(depart, 1u) == static_cast<uint32_t>(p.gsplit) - 1) {
+    // the last CTA of the tile to leave resets the counters for the next call
+    *arrive = 0u;
+    *depart = 0u;
+  }
+}
+
 template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -286,15 +362,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if constexpr (SPLIT > 1) cluster_sync_all();
   const uint32_t tmem_base = *tmem_slot;
+
+  // split-K: one tile per CTA (t_step ends the tile loop after it)
+  const uint32_t rank = SPLIT > 1 ? cluster_ctarank()
+                        : SPLIT == kGlobalSplit ? blockIdx.x % static_cast<uint32_t>(p.gsplit) : 0u;
+  const int t_first = SPLIT > 1 ? static_cast<int>(blockIdx.x) / SPLIT
+                      : SPLIT == kGlobalSplit ? static_cast<int>(blockIdx.x) / p.gsplit
+                                              : static_cast<int>(blockIdx.x);
+  const int t_step = SPLIT != 1 ? p.num_tiles : static_cast<int>(gridDim.x);
+
+  if constexpr (KIND == kDense) {
+    // start the first stages' HBM reads into L2 before waiting for the
+    // previous kernel; the loads after the wait then find them in L2
+    if ((warp == 0 || warp == 3) && lane < kIssuersPerWarp && t_first < p.num_tiles) {
+      const int me = (warp == 3 ? kIssuersPerWarp : 0) + lane;
+      const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t_first, rank, false);
+      for (int i = me; i < STAGES && T.kb0 + i < T.kb1; i += kIssuers) {
+        const int kb = T.kb0 + i;
+        tma_prefetch_3d(kSwap ? &tmB : &tmA, kb * 128, kSwap ? T.n0 : T.m0, 0);
+        tma_prefetch_3d(kSwap ? &tmA : &tmB, kb * 128, kSwap ? T.m0 : T.n0, 0);
+      }
+    }
+  }
   // inputs may be written by the previous kernel in the stream: wait for it
   // (a no-op without a programmatic dependency), then let the next one start
   // its own prologue
   grid_dependency_wait();
   if (threadIdx.x == 0) grid_launch_dependents();
-
-  const uint32_t rank = SPLIT > 1 ? cluster_ctarank() : 0u;
-  const int t_first = SPLIT > 1 ? static_cast<int>(blockIdx.x) / SPLIT : static_cast<int>(blockIdx.x);
-  const int t_step = SPLIT > 1 ? p.num_tiles : static_cast<int>(gridDim.x);
   constexpr uint32_t kStageTx = L::kLaneBytes + L::kColBytes + L::kSaFloats * 4;
 
   if (warp < 4) {
@@ -469,7 +563,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
 
       const long drow0 = KIND == kMasked ? static_cast<long>(T.g) * p.M : 0;
-      if constexpr (SPLIT > 1) {
+      if constexpr (SPLIT == kGlobalSplit) {
+        // partial sums to the workspace, column-major per tile slot so that a
+        // warp's 32 rows of one column are 128 contiguous bytes
+        float* slot = p.ws + (static_cast<long>(t) * p.gsplit + rank) * (BNC * 128);
+#pragma unroll
+        for (int c = 0; c < kCW; ++c) slot[(wg * kCW + c) * 128 + row] = acc[c];
+      } else if constexpr (SPLIT > 1) {
         // store this CTA's partial columns into the shared memory of the CTA
         // that reduces them (slot = this CTA's rank); the reduction follows
         // the cluster barrier after the role loops
@@ -513,6 +613,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncwarp();
+  if constexpr (SPLIT == kGlobalSplit) {
+    if (warp >= 4) global_split_reduce<BNC, KIND>(p, t_first, rank, abort_flag);
+  }
   if constexpr (SPLIT > 1) {
     // all partials of this cluster's tile are in place after the barrier;
     // the warpgroup whose columns this CTA owns adds them in rank order
