@@ -488,3 +488,125 @@ int fp8g_last_variant(void) { return t_last_variant; }
 int fp8g_version(void) { return 100; }
 
 }  // extern "C"
+
+// ===========================================================================
+// fp8_gemm_nt_no_alloc: the dense GEMM for callers that must not allocate
+// device memory.
+//
+// Some callers cannot call cudaMalloc at the point where they run a GEMM: an
+// engine that hands out all device memory from its own fixed pool, code that
+// runs while another component is capturing a CUDA graph (an allocation
+// there would break the capture), or a runtime that forbids allocations
+// after start-up so that its memory footprint is known in advance.  The
+// regular fp8_gemm_nt allocates its split-K workspace (about 4.7 MB) on the
+// first decode-shaped call of a device.  This entry point runs the same
+// split-K kernel with its scratch in a statically sized array that the
+// library carries in its own device image instead.
+// ===========================================================================
+namespace {
+
+// Scratch of the static variant: 160 tile slots of 64 x 128 FP32 partial sums,
+// then 2 counters per tile.  Every GPU that loads the library holds it until
+// the process exits.
+constexpr int kNoAllocSlots = 160;
+constexpr size_t kNoAllocPartialBytes = static_cast<size_t>(kNoAllocSlots) * 64 * 128 * sizeof(float);
+constexpr size_t kNoAllocCounterBytes = static_cast<size_t>(kNoAllocSlots) * 2 * sizeof(uint32_t);
+
+static __device__ __align__(256) unsigned char g_no_alloc_scratch[kNoAllocPartialBytes + kNoAllocCounterBytes];
+
+std::mutex g_no_alloc_mu;
+void* g_no_alloc_ptr[kMaxDevices] = {};  // device address of g_no_alloc_scratch, per device
+
+// Device address of the static scratch on the current device.  The symbol's
+// name in host code only stands for the array; the device address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+int no_alloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_no_alloc_mu);
+  if (!g_no_alloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_no_alloc_scratch) != cudaSuccess || !ptr) {
+      (void)cudaGetLastError();
+      return FP8G_ERR_CUDA;
+    }
+    g_no_alloc_ptr[dev] = ptr;
+  }
+  *out = g_no_alloc_ptr[dev];
+  return FP8G_OK;
+}
+
+}  // namespace
+
+extern "C" int fp8_gemm_nt_no_alloc(const uint8_t* A, const float* sa, int ld_sa, const uint8_t* B,
+                                    const float* sb, uint16_t* D, int M, int N, int K, cudaStream_t stream) {
+  int rc = check_shapes(M, N, K, ld_sa);
+  if (rc) return rc;
+  if (M == 0 || N == 0) return FP8G_OK;
+  if ((rc = check_ptrs(A, sa, B, sb, D))) return rc;
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev))) return rc;
+  int dev_id = 0;
+  if (cudaGetDevice(&dev_id) != cudaSuccess) return FP8G_ERR_CUDA;
+
+  // tiles of 128 rows of B x 64 rows of A; K split over `gsplit` CTAs per tile
+  const Variant& V = kVariants[V_DENSE_GSPLIT];
+  const int KB = K / 128, NB = (N + 127) / 128;
+  const int n_tiles = NB, m_tiles = (M + 63) / 64;
+  const long tiles = static_cast<long>(n_tiles) * m_tiles;
+  if (tiles > kNoAllocSlots || tiles > dev->sms) return FP8G_ERR_UNSUPPORTED;  // scratch or GPU too small
+  const int gsplit = std::min(gsplit_for(dev, static_cast<int>(tiles), KB), kNoAllocSlots / static_cast<int>(tiles));
+  if (gsplit < 1) return FP8G_ERR_UNSUPPORTED;
+  if ((rc = prepare_variant(dev, V_DENSE_GSPLIT))) return rc;
+  void* scratch = nullptr;
+  if ((rc = no_alloc_scratch(dev_id, &scratch))) return rc;
+
+  Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.KB = KB;
+  p.NB = NB;
+  p.G = 1;
+  p.n_tiles = n_tiles;
+  p.m_tiles = m_tiles;
+  p.num_tiles = static_cast<int>(tiles);
+  p.sb = sb;
+  p.D = D;
+  p.gsplit = gsplit;
+  p.ws = static_cast<float*>(scratch);
+  p.sync = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(scratch) + kNoAllocPartialBytes);
+  // the counters of this call start at zero even if an earlier call gave up
+  // half-way; the partial sums are always written before they are read
+  if (cudaMemsetAsync(p.sync, 0, static_cast<size_t>(2) * p.num_tiles * sizeof(uint32_t), stream) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FP8G_ERR_CUDA;
+  }
+
+  CUtensorMap tmA, tmB, tmSA;
+  rc = encode3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, 1, (uint64_t)K, (uint64_t)K * M, 128, V.bnc,
+                CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!rc)
+    rc = encode3d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, 1, (uint64_t)K, (uint64_t)K * N, 128, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!rc)
+    rc = encode3d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sa, M, KB, 1, (uint64_t)ld_sa * 4, (uint64_t)ld_sa * 4 * KB,
+                  V.bnc, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(p.num_tiles * p.gsplit, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = V.smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  void* args[] = {&tmA, &tmB, &tmSA, &p};
+  if (cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(V.fn), args) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FP8G_ERR_CUDA;
+  }
+  t_last_variant = V_DENSE_GSPLIT;
+  return FP8G_OK;
+}

@@ -28,6 +28,8 @@ lib.m_grouped_fp8_gemm_nt_contiguous.restype = _I
 lib.m_grouped_fp8_gemm_nt_contiguous.argtypes = [_P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P]
 lib.m_grouped_fp8_gemm_nt_masked.restype = _I
 lib.m_grouped_fp8_gemm_nt_masked.argtypes = [_P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
+lib.fp8_gemm_nt_no_alloc.restype = _I
+lib.fp8_gemm_nt_no_alloc.argtypes = [_P, _P, _I, _P, _P, _P, _I, _I, _I, _P]
 lib.fp8g_status_string.restype = C.c_char_p
 lib.fp8g_status_string.argtypes = [_I]
 lib.fp8g_get_device_error.restype = _I
@@ -138,4 +140,22 @@ def m_grouped_fp8_gemm_nt_masked(A, sa, B, sb, masked_m, expected_m, D=None, str
     _check(lib.m_grouped_fp8_gemm_nt_masked(_ptr(A), _ptr(sa), sa.shape[2], _ptr(B), _ptr(sb), _ptr(D),
                                             _ptr(masked_m), G, Mmax, N, K, int(expected_m),
                                             _stream(stream)), "m_grouped_fp8_gemm_nt_masked")
+    return D
+
+
+def fp8_gemm_nt_no_alloc(A, sa, B, sb, D=None, stream=None):
+    """Dense GEMM like fp8_gemm_nt, for callers that must not allocate device
+    memory while they run it (the library keeps this path's split-K scratch in
+    a fixed array of its own).  Decode shapes only: at most 160 tiles of 128
+    rows of B by 64 rows of A.  Pass D to avoid the output allocation here;
+    calls that overlap on the GPU share the scratch and must be ordered."""
+    M, K = A.shape
+    N = B.shape[0]
+    _dev(A, torch.uint8, "A"), _dev(B, torch.uint8, "B")
+    _dev(sa, torch.float32, "sa"), _dev(sb, torch.float32, "sb")
+    if D is None:
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _dev(D, torch.bfloat16, "D")
+    _check(lib.fp8_gemm_nt_no_alloc(_ptr(A), _ptr(sa), sa.shape[1], _ptr(B), _ptr(sb), _ptr(D), M, N, K,
+                                    _stream(stream)), "fp8_gemm_nt_no_alloc")
     return D

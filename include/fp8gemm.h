@@ -113,6 +113,35 @@ int m_grouped_fp8_gemm_nt_masked(const uint8_t *A, const float *sa, int ld_sa,
                                  int G, int Mmax, int N, int K, int expected_m,
                                  cudaStream_t stream);
 
+/*
+ * Dense NT GEMM that allocates no device memory (the method's pages have no
+ * counterpart: this serves callers that cannot allocate).
+ *
+ * Same operation, layouts, requirements and errors as fp8_gemm_nt.  It exists
+ * for callers that must not call cudaMalloc when they run a GEMM: an engine
+ * that hands out all device memory from its own pool, or code that runs while
+ * a CUDA graph is being captured.  fp8_gemm_nt allocates a split-K workspace
+ * (about 4.7 MB) on the first decode-shaped call of each device; this entry
+ * point instead keeps its scratch (the split-K partial sums and two counters
+ * per tile) in a fixed array of 5 MiB + 1.25 KiB inside the library, which
+ * every GPU that loads the library holds until the process exits.
+ *  - It always runs the split-K kernel for decode shapes: tiles of 128 rows of
+ *    B by 64 rows of A, K split over several CTAs per tile.  A shape with more
+ *    than 160 such tiles (ceil(N/128) * ceil(M/64)), or more tiles than the GPU
+ *    has SMs, needs more scratch than the array holds and returns
+ *    FP8G_ERR_UNSUPPORTED without launching anything.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call enqueues a small memset of its counters and one kernel on
+ *    `stream`; it calls no cudaMalloc, cudaFree or other allocating routine.
+ *  - All calls share the one array: calls whose executions overlap on the
+ *    GPU (on different streams, or on one stream without ordering between
+ *    them) race on it and give wrong results.  Order such calls.
+ */
+int fp8_gemm_nt_no_alloc(const uint8_t *A, const float *sa, int ld_sa,
+                         const uint8_t *B, const float *sb,
+                         uint16_t *D, int M, int N, int K, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *fp8g_status_string(int status);
 
