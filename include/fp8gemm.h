@@ -36,9 +36,9 @@
  *      A, B, sa, D 16-byte aligned; sb, m_indices, masked_m 4-byte aligned.
  *    M == 0 or N == 0 (or G == 0) is a no-op that returns FP8G_OK.
  *  - The call enqueues kernels on `stream` and returns without waiting.  It
- *    never synchronises and never reads device memory on the host, so it can
- *    be captured in a CUDA graph.  D is complete when the stream reaches
- *    that point.
+ *    never reads device memory on the host, so it can be captured in a CUDA
+ *    graph.  D is complete when the stream reaches that point.  The one
+ *    exception to "never waits": see fp8_gemm_nt's workspace below.
  *  - Errors found on the host come back as the return value; nothing is
  *    launched then.  Errors found by the kernel (a bad m_indices entry, a
  *    masked_m above Mmax, a pipeline wait that timed out) are recorded in a
@@ -75,6 +75,12 @@ enum fp8g_status {
  * Dense NT GEMM (GeekNews page, "일반 GEMM 성능 (Dense 모델)").
  *   A [M,K], sa [K/128][ld_sa], B [N,K], sb [ceil(N/128)][K/128], D [M,N].
  * Every element of D is written.
+ * Decode shapes (M <= 64) split K over several CTAs per tile.  The first such
+ * call on a device allocates a split-K workspace of about 4.7 MB (kept until
+ * the process exits) and synchronises the device once.  If that first call
+ * happens while `stream` is being captured, nothing is allocated and the call
+ * uses a split-K kernel without a workspace (same results).  Callers that
+ * cannot allocate at all use fp8_gemm_nt_no_alloc.
  */
 int fp8_gemm_nt(const uint8_t *A, const float *sa, int ld_sa,
                 const uint8_t *B, const float *sb,
