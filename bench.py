@@ -143,6 +143,12 @@ class ClockSampler:
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    @classmethod
+    def disabled(cls):
+        obj = cls.__new__(cls)
+        obj.samples, obj.proc = [], None
+        return obj
+
     def _read(self):
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
@@ -321,7 +327,7 @@ def run_ours(args, rank: int, world: int) -> None:
     timed_graph, evs = capture(args.steps, args.warmup, args.per_launch_events)
 
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    sampler = ClockSampler(gpu_id)
+    sampler = ClockSampler(gpu_id) if not args.no_clocks else ClockSampler.disabled()
 
     def timed_region():
         # graph.replay() launches on torch's current stream: make it `stream`,
@@ -332,6 +338,10 @@ def run_ours(args, rank: int, world: int) -> None:
             while time.time() - soak_t0 < 0.6:
                 warm_graph.replay()
                 torch.cuda.synchronize(dev)
+            # a graph's first replay also uploads it to the device; do that
+            # outside the timed region
+            timed_graph.replay()
+            torch.cuda.synchronize(dev)
             warm_graph.replay()
             start = torch.cuda.Event(enable_timing=True)
             end = torch.cuda.Event(enable_timing=True)
@@ -461,6 +471,7 @@ def main() -> int:
     ap.add_argument("--variant", type=int, default=None, help="force a kernel variant (tuning)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi clocks (diagnostic)")
     ap.add_argument("--per-launch-events", action="store_true",
                     help="record an event between launches (diagnostic; prevents launch overlap)")
     args = ap.parse_args()

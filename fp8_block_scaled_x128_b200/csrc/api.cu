@@ -31,11 +31,11 @@ struct Variant {
   int smem;
 };
 
-template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT>
+template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int MINB = 1>
 Variant make_variant(const char* name) {
-  using L = Layout<kSwap, BNC, STAGES, SPLIT>;
+  using L = Layout<kSwap, BNC, STAGES, SPLIT, MINB>;
   return Variant{name, KIND, kSwap, BNC, STAGES, SPLIT, L::kRegSplit,
-                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT>, L::kSmemAlloc};
+                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT, MINB>, L::kSmemAlloc};
 }
 
 // "nlanes": TMEM lanes are rows of B (small M); "mlanes": lanes are rows of A.
@@ -55,6 +55,8 @@ const Variant kVariants[] = {
     make_variant<false, 256, 4, kContiguous, 1>("contiguous_mlanes_bn256_st4"),
     make_variant<false, 256, 4, kMasked, 1>("masked_mlanes_bn256_st4"),
     make_variant<true, 64, 8, kDense, kGlobalSplit>("dense_nlanes_bn64_st8_gsplit"),
+    make_variant<true, 64, 8, kDense, kGlobalSplitPartials>("dense_nlanes_bn64_st8_gsplit_2k"),
+    make_variant<true, 64, 4, kDense, kGlobalSplitPartials, 2>("dense_nlanes_bn64_st4_gsplit_2k_x2"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
@@ -73,6 +75,8 @@ enum : int {
   V_CONTIG_M256 = 12,
   V_MASKED_M256 = 13,
   V_DENSE_GSPLIT = 14,
+  V_DENSE_GSPLIT2K = 15,
+  V_DENSE_GSPLIT2K_X2 = 16,
 };
 
 std::atomic<int> g_override{-1};
@@ -298,7 +302,7 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   p.sb = P.sb;
   p.D = P.D;
   if (p.num_tiles <= 0) return FP8G_OK;
-  if (V.split == kGlobalSplit) {
+  if (V.split < 0) {
     p.gsplit = gsplit_for(dev, p.num_tiles, KB);
     if (p.gsplit < 1 || p.num_tiles * p.gsplit > dev->sms) return FP8G_ERR_UNSUPPORTED;
     if ((rc = ensure_workspace(dev, stream))) return rc;
@@ -339,8 +343,8 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
     attr[nattr].val.clusterDim.z = 1;
     ++nattr;
     cfg.gridDim = dim3(p.num_tiles * V.split, 1, 1);
-  } else if (V.split == kGlobalSplit) {
-    cfg.gridDim = dim3(p.num_tiles * p.gsplit, 1, 1);
+  } else if (V.split < 0) {
+    cfg.gridDim = dim3(p.gsplit, p.n_tiles, p.m_tiles);
   } else {
     cfg.gridDim = dim3(std::min(p.num_tiles, dev->sms), 1, 1);
   }
@@ -350,6 +354,25 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   if (cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(V.fn), args) != cudaSuccess) {
     (void)cudaGetLastError();
     return FP8G_ERR_CUDA;
+  }
+  if (V.split == kGlobalSplitPartials) {
+    // the sum of the partials, one thread per output element
+    cudaLaunchConfig_t rc_cfg = {};
+    cudaLaunchAttribute rc_attr[1];
+    const long outputs = static_cast<long>(p.num_tiles) * V.bnc * 128;
+    rc_cfg.gridDim = dim3(static_cast<unsigned>(std::min<long>((outputs + 255) / 256, 4L * dev->sms)), 1, 1);
+    rc_cfg.blockDim = dim3(256, 1, 1);
+    rc_cfg.stream = stream;
+    rc_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    rc_attr[0].val.programmaticStreamSerializationAllowed = 1;
+    rc_cfg.attrs = rc_attr;
+    rc_cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    void* rargs[] = {&p};
+    if (cudaLaunchKernelExC(&rc_cfg, reinterpret_cast<const void*>(&splitk_reduce_kernel<64>), rargs) !=
+        cudaSuccess) {
+      (void)cudaGetLastError();
+      return FP8G_ERR_CUDA;
+    }
   }
   t_last_variant = v;
   return FP8G_OK;
@@ -371,9 +394,9 @@ int select_variant(const Problem& P, DeviceInfo* dev, cudaStream_t stream) {
     // co-resident and that leaves each CTA at least 4 K-blocks.
     const int nt = (P.N + 127) / 128;
     const int kb = P.K / 128;
-    if (gsplit_for(dev, nt, kb) >= 2 && prepare_variant(dev, V_DENSE_GSPLIT) == FP8G_OK &&
+    if (gsplit_for(dev, nt, kb) >= 2 && prepare_variant(dev, V_DENSE_GSPLIT2K) == FP8G_OK &&
         ensure_workspace(dev, stream) == FP8G_OK)
-      return V_DENSE_GSPLIT;
+      return V_DENSE_GSPLIT2K;
     for (int v : {V_DENSE_SPLIT, V_DENSE_SPLIT4, V_DENSE_SPLIT2}) {
       const int split = kVariants[v].split;
       if (kb < 4 * split || nt * split > dev->sms) continue;
@@ -594,7 +617,7 @@ extern "C" int fp8_gemm_nt_no_alloc(const uint8_t* A, const float* sa, int ld_sa
 
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3(p.num_tiles * p.gsplit, 1, 1);
+  cfg.gridDim = dim3(p.gsplit, p.n_tiles, p.m_tiles);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = V.smem;
   cfg.stream = stream;

@@ -103,8 +103,12 @@ struct Params {
   uint32_t* sync;
 };
 
-// SPLIT template value selecting the global-memory split-K (count at run time)
+// SPLIT template values selecting the global-memory split-K (count at run
+// time): kGlobalSplit reduces inside the kernel after a per-tile arrival
+// count; kGlobalSplitPartials only stores the partials and leaves the sum to
+// splitk_reduce_kernel, launched next on the same stream.
 constexpr int kGlobalSplit = -1;
+constexpr int kGlobalSplitPartials = -2;
 constexpr int kMaxGSplit = 16;  // the host never picks more
 
 constexpr int pow2_at_least(int x, int lo) {
@@ -113,12 +117,16 @@ constexpr int pow2_at_least(int x, int lo) {
   return p;
 }
 
-template <bool kSwap, int BNC, int STAGES, int SPLIT>
+// MINB: CTAs that must fit on one SM together (2 lets the next launch's
+// CTAs start their prologue beside a running CTA: half the TMEM and shared
+// memory, and at most 85 registers per thread).
+template <bool kSwap, int BNC, int STAGES, int SPLIT, int MINB = 1>
 struct Layout {
   static constexpr int kLaneBytes = 128 * 128;   // 128 rows x 128 e4m3 (one K-block)
   static constexpr int kColBytes = BNC * 128;
   static constexpr int kSaFloats = kSwap ? BNC : 128;  // sa slice: the tile's m-extent
-  static constexpr int kNBuf = 512 / BNC < 8 ? 512 / BNC : 8;  // TMEM partial buffers
+  static constexpr int kTmemBudget = 512 / MINB;
+  static constexpr int kNBuf = kTmemBudget / BNC < 8 ? kTmemBudget / BNC : 8;  // TMEM partial buffers
   static constexpr int kTmemCols = pow2_at_least(kNBuf * BNC, 32);
   static constexpr int kCW = BNC / 2;                  // columns per promotion warpgroup
   static constexpr bool kRegSplit = kCW > 64;          // 128 accumulators per thread
@@ -142,9 +150,10 @@ struct Layout {
   static_assert(kColBytes % 1024 == 0, "column tile rows must be a multiple of 8");
   static_assert(SPLIT <= 1 || (kSwap && BNC % SPLIT == 0 && kCW % kCPD == 0 && kCPD % 4 == 0),
                 "cluster split-K layout");
-  static_assert(SPLIT != kGlobalSplit || kSwap, "global split-K is for the n-lanes orientation");
+  static_assert(SPLIT >= 1 || kSwap, "global split-K is for the n-lanes orientation");
   static_assert(!kRegSplit || !kSwap, "the register split is for the m-lanes orientation");
-  static_assert(kSmemAlloc <= 232448, "shared memory");
+  static_assert(kSmemAlloc <= 232448 && kSmemAlloc * MINB <= 231424, "shared memory");
+  static_assert(kNBuf >= 2, "TMEM buffers");
 };
 
 // Register budget of the BNC = 256 variants: 384 threads launch with 168
@@ -176,7 +185,9 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int t, uint32_t rank, 
     T.kb1 = static_cast<int>((static_cast<long>(p.KB) * (rank + 1)) / ns);
   }
   if constexpr (KIND == kDense) {
-    const int nt = t % p.n_tiles, mt = t / p.n_tiles;
+    // global split-K: the grid carries the tile coordinates (t == mt*n_tiles + nt)
+    const int nt = SPLIT < 0 ? static_cast<int>(blockIdx.y) : t % p.n_tiles;
+    const int mt = SPLIT < 0 ? static_cast<int>(blockIdx.z) : t / p.n_tiles;
     T.m0 = mt * kMExt;
     T.n0 = nt * kNExt;
     T.mvalid = min(kMExt, p.M - T.m0);
@@ -305,11 +316,11 @@ __device__ __forceinline__ void global_split_reduce(const Params& p, int tile, u
   }
 }
 
-template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int MINB = 1>
+__global__ void __launch_bounds__(kThreads, MINB)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSA, const Params p) {
-  using L = Layout<kSwap, BNC, STAGES, SPLIT>;
+  using L = Layout<kSwap, BNC, STAGES, SPLIT, MINB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -363,27 +374,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (SPLIT > 1) cluster_sync_all();
   const uint32_t tmem_base = *tmem_slot;
 
-  // split-K: one tile per CTA (t_step ends the tile loop after it)
-  const uint32_t rank = SPLIT > 1 ? cluster_ctarank()
-                        : SPLIT == kGlobalSplit ? blockIdx.x % static_cast<uint32_t>(p.gsplit) : 0u;
+  // split-K: one tile per CTA (t_step ends the tile loop after it).  The
+  // global split-K grid is (rank, N-tile, M-tile), so no division is needed.
+  const uint32_t rank = SPLIT > 1 ? cluster_ctarank() : SPLIT < 0 ? blockIdx.x : 0u;
   const int t_first = SPLIT > 1 ? static_cast<int>(blockIdx.x) / SPLIT
-                      : SPLIT == kGlobalSplit ? static_cast<int>(blockIdx.x) / p.gsplit
-                                              : static_cast<int>(blockIdx.x);
+                      : SPLIT < 0 ? static_cast<int>(blockIdx.z * gridDim.y + blockIdx.y)
+                                  : static_cast<int>(blockIdx.x);
   const int t_step = SPLIT != 1 ? p.num_tiles : static_cast<int>(gridDim.x);
 
-  if constexpr (KIND == kDense) {
-    // start the first stages' HBM reads into L2 before waiting for the
-    // previous kernel; the loads after the wait then find them in L2
-    if ((warp == 0 || warp == 3) && lane < kIssuersPerWarp && t_first < p.num_tiles) {
-      const int me = (warp == 3 ? kIssuersPerWarp : 0) + lane;
-      const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t_first, rank, false);
-      for (int i = me; i < STAGES && T.kb0 + i < T.kb1; i += kIssuers) {
-        const int kb = T.kb0 + i;
-        tma_prefetch_3d(kSwap ? &tmB : &tmA, kb * 128, kSwap ? T.n0 : T.m0, 0);
-        tma_prefetch_3d(kSwap ? &tmA : &tmB, kb * 128, kSwap ? T.m0 : T.n0, 0);
-      }
-    }
-  }
   // inputs may be written by the previous kernel in the stream: wait for it
   // (a no-op without a programmatic dependency), then let the next one start
   // its own prologue
@@ -563,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
 
       const long drow0 = KIND == kMasked ? static_cast<long>(T.g) * p.M : 0;
-      if constexpr (SPLIT == kGlobalSplit) {
+      if constexpr (SPLIT < 0) {
         // partial sums to the workspace, column-major per tile slot so that a
         // warp's 32 rows of one column are 128 contiguous bytes
         float* slot = p.ws + (static_cast<long>(t) * p.gsplit + rank) * (BNC * 128);
@@ -658,6 +656,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+// Second kernel of the two-kernel split-K: D[m0 + c, n0 + r] = bf16(sum over
+// ranks, in rank order, of the partials ws[tile][rank][c][r]).  Launched after
+// the GEMM kernel on the same stream (programmatic dependent launch: it waits
+// for the GEMM kernel's partials, and lets the next kernel start its
+// prologue early).  One thread per output element, grid-stride.
+template <int BNC>
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const Params p) {
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
+  const long total = static_cast<long>(p.num_tiles) * BNC * 128;
+  const long stride = static_cast<long>(gridDim.x) * blockDim.x;
+  for (long e = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const int tile = static_cast<int>(e / (BNC * 128));
+    const int c = static_cast<int>((e / 128) % BNC);
+    const int r = static_cast<int>(e % 128);
+    const int m = (tile / p.n_tiles) * BNC + c;
+    const int n = (tile % p.n_tiles) * 128 + r;
+    if (m >= p.M || n >= p.N) continue;
+    const float* src = p.ws + static_cast<long>(tile) * p.gsplit * (BNC * 128) + c * 128 + r;
+    float v[kMaxGSplit];
+#pragma unroll
+    for (int i = 0; i < kMaxGSplit; ++i) v[i] = i < p.gsplit ? __ldcg(src + static_cast<long>(i) * (BNC * 128)) : 0.f;
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxGSplit; ++i) sum += v[i];
+    p.D[static_cast<long>(m) * p.N + n] = static_cast<uint16_t>(pack_bf16x2(sum, 0.f) & 0xFFFFu);
   }
 }
 
