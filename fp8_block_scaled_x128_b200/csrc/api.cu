@@ -299,6 +299,8 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   p.num_tiles = p.n_tiles * p.m_tiles * (P.kind == kMasked ? P.G : 1);
   p.m_indices = P.kind == kContiguous ? P.idx : nullptr;
   p.masked_m = P.kind == kMasked ? P.idx : nullptr;
+  p.sa = P.sa;
+  p.ld_sa = P.ld_sa;
   p.sb = P.sb;
   p.D = P.D;
   if (p.num_tiles <= 0) return FP8G_OK;
@@ -387,7 +389,13 @@ int select_variant(const Problem& P, DeviceInfo* dev, cudaStream_t stream) {
   };
   if (P.kind == kContiguous)
     return wide(V_CONTIG_M256, V_CONTIG_M128, static_cast<long>(P.M / 128) * ((P.N + 255) / 256));
-  if (P.kind == kMasked) return P.expected_m > 0 && P.expected_m <= 64 ? V_MASKED_N64 : V_MASKED_N128;
+  if (P.kind == kMasked) {
+    if (P.expected_m > 0 && P.expected_m <= 64) return V_MASKED_N64;
+    // B streams once per 128 rows of a group's A: m-lanes tiles read it the
+    // fewest times; count the tiles the typical group fills
+    const long m_blocks = (std::max(P.expected_m, 1) + 127) / 128;
+    return wide(V_MASKED_M256, V_MASKED_M128, static_cast<long>(P.G) * m_blocks * ((P.N + 255) / 256));
+  }
   if (P.M <= 64) {
     // decode shapes: few 128-row tiles of B.  Split K over a cluster so that
     // many SMs stream B; take the largest split whose clusters are all
@@ -592,6 +600,8 @@ extern "C" int fp8_gemm_nt_no_alloc(const uint8_t* A, const float* sa, int ld_sa
   p.n_tiles = n_tiles;
   p.m_tiles = m_tiles;
   p.num_tiles = static_cast<int>(tiles);
+  p.sa = sa;
+  p.ld_sa = ld_sa;
   p.sb = sb;
   p.D = D;
   p.gsplit = gsplit;

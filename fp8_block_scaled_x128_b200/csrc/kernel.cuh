@@ -92,6 +92,8 @@ struct Params {
   int num_tiles;
   const int32_t* m_indices;
   const int32_t* masked_m;
+  const float* sa;  // [G][KB][ld_sa] (masked) or [KB][ld_sa]
+  int ld_sa;
   const float* sb;  // [G][NB][KB]
   uint16_t* D;
   // global split-K (SPLIT == kGlobalSplit): K is split over `gsplit` CTAs per
@@ -124,7 +126,7 @@ template <bool kSwap, int BNC, int STAGES, int SPLIT, int MINB = 1>
 struct Layout {
   static constexpr int kLaneBytes = 128 * 128;   // 128 rows x 128 e4m3 (one K-block)
   static constexpr int kColBytes = BNC * 128;
-  static constexpr int kSaFloats = kSwap ? BNC : 128;  // sa slice: the tile's m-extent
+  static constexpr int kSaFloats = kSwap ? BNC : 0;  // sa slice (n-lanes only): the tile's m-extent
   static constexpr int kTmemBudget = 512 / MINB;
   static constexpr int kNBuf = kTmemBudget / BNC < 8 ? kTmemBudget / BNC : 8;  // TMEM partial buffers
   static constexpr int kTmemCols = pow2_at_least(kNBuf * BNC, 32);
@@ -348,7 +350,8 @@ __global__ void __launch_bounds__(kThreads, MINB)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1 + kPromoWarps);  // MMA commit + promotion warps (they read sa)
+      // MMA commit, plus the promotion warps where they read the stage's sa slice
+      mbar_init(empty_bar(s), kSwap ? 1 + kPromoWarps : 1);
     }
     for (int b = 0; b < L::kNBuf; ++b) {
       mbar_init(tfull_bar(b), 1);
@@ -420,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
             tma_load_3d(lane_tile(s), &tmA, full_bar(s), kb * 128, T.m0, ga);
             tma_load_3d(col_tile(s), &tmB, full_bar(s), kb * 128, T.n0, gb);
           }
-          tma_load_3d(sa_slice(s), &tmSA, full_bar(s), T.m0, kb, ga);
+          if constexpr (kSwap) tma_load_3d(sa_slice(s), &tmSA, full_bar(s), T.m0, kb, ga);
         }
       }
       // drain: every load this thread issued must land before the CTA exits
@@ -488,54 +491,104 @@ __global__ void __launch_bounds__(kThreads, MINB)
       for (int c = 0; c < kCW; ++c) acc[c] = 0.f;
       // column chunks of 32 that hold valid output (kSwap: columns are rows of A)
       const int live = kSwap ? min(kCW, max(0, T.mvalid - wg * kCW)) : kCW;
-      // the sb row of this thread's columns, 32 K-blocks per register (lane i
-      // holds K-block kb0 + 32j + i), the next chunk loaded one chunk ahead
+      // the sb row of this thread's columns (n-lanes: 32 K-blocks per
+      // register, lane i holding K-block kb0 + 32j + i, the next 32 loaded
+      // one chunk ahead and broadcast with a shuffle)
       const int nb = min((kSwap ? T.n0 : T.n0 + wg * kCW) / 128, p.NB - 1);
       const float* sbp = p.sb + (static_cast<long>(T.g) * p.NB + nb) * p.KB;
-      float sb_cur = T.kb0 + lane < T.kb1 ? __ldg(sbp + T.kb0 + lane) : 0.f;
-      float sb_nxt = T.kb0 + 32 + lane < T.kb1 ? __ldg(sbp + T.kb0 + 32 + lane) : 0.f;
-      for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1u;
-        const int b = it % L::kNBuf;
-        const uint32_t tph = (it / L::kNBuf) & 1u;
-        const int i32 = (kb - T.kb0) & 31;
-        if (i32 == 0 && kb != T.kb0) {
-          sb_cur = sb_nxt;
-          sb_nxt = kb + 32 + lane < T.kb1 ? __ldg(sbp + kb + 32 + lane) : 0.f;
+      // chunks of 32 columns, loaded two at a time (64 staging registers)
+      constexpr int kChunks = kCW / 32;
+      constexpr int kGroup = kChunks < 2 ? kChunks : 2;
+      if constexpr (!kSwap) {
+        // m-lanes: one scale per thread and K-block, sa[kb][m0 + row] *
+        // sb[g][nb][kb], read from global memory two K-blocks ahead, so the
+        // loop waits on nothing but the partial in TMEM
+        const bool row_in = T.m0 + row < p.M;
+        const float* sap = p.sa + (KIND == kMasked ? static_cast<long>(T.g) * p.KB * p.ld_sa : 0L) + T.m0 + row;
+        auto sa_at = [&](int kb) { return row_in && kb < T.kb1 ? __ldg(sap + static_cast<long>(kb) * p.ld_sa) : 0.f; };
+        auto sb_at = [&](int kb) { return kb < T.kb1 ? __ldg(sbp + kb) : 0.f; };
+        float sa0 = sa_at(T.kb0), sa1 = sa_at(T.kb0 + 1);
+        float sb0 = sb_at(T.kb0), sb1 = sb_at(T.kb0 + 1);
+        for (int kb = T.kb0; ok && kb < T.kb1; kb += 2) {
+          const float sc2[2] = {sa0 * sb0, sa1 * sb1};
+          sa0 = sa_at(kb + 2);
+          sa1 = sa_at(kb + 3);
+          sb0 = sb_at(kb + 2);
+          sb1 = sb_at(kb + 3);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            if (kb + u >= T.kb1) break;
+            const int b = it % L::kNBuf;
+            const uint32_t tph = (it / L::kNBuf) & 1u;
+            if (!__all_sync(0xffffffffu, wait_phase(tfull_bar(b), tph, abort_flag))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                   static_cast<uint32_t>(b * BNC + wg * kCW);
+#pragma unroll
+            for (int j0 = 0; j0 < kChunks; j0 += kGroup) {
+              uint32_t r[kGroup][32];
+#pragma unroll
+              for (int j = 0; j < kGroup; ++j) tmem_ld_32x32b_x32(taddr + 32 * (j0 + j), r[j]);
+              tmem_ld_wait_bind(r[0]);
+#pragma unroll
+              for (int j = 1; j < kGroup; ++j) bind_after_wait(r[j]);
+#pragma unroll
+              for (int j = 0; j < kGroup; ++j) {
+                float* a = acc + 32 * (j0 + j);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
+              }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(b));
+            ++it;
+          }
         }
-        const float s_b = __shfl_sync(0xffffffffu, sb_cur, i32);
-        // the stage's sa slice is read below: wait for its TMA as well
-        bool w = wait_phase(tfull_bar(b), tph, abort_flag);
-        w = w && wait_phase(full_bar(s), ph, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
-                               static_cast<uint32_t>(b * BNC + wg * kCW);
-        // this thread's scale: sa[m0 + row, kb] * sb[nb, kb] (m-lanes), or
-        // per column sa[m0 + c, kb] * sb[nb, kb] (n-lanes)
-        const float sc_row = kSwap ? 0.f : sa_f[s * L::kSaFloats + row] * s_b;
-        // chunks of 32 columns, loaded two at a time (64 staging registers)
-        constexpr int kChunks = kCW / 32;
-        constexpr int kGroup = kChunks < 2 ? kChunks : 2;
+      } else {
+        // n-lanes: the scale varies per column (sa slice of the stage) and
+        // is uniform over the lanes for sb (broadcast from a register)
+        float sb_cur = T.kb0 + lane < T.kb1 ? __ldg(sbp + T.kb0 + lane) : 0.f;
+        float sb_nxt = T.kb0 + 32 + lane < T.kb1 ? __ldg(sbp + T.kb0 + 32 + lane) : 0.f;
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          const int b = it % L::kNBuf;
+          const uint32_t tph = (it / L::kNBuf) & 1u;
+          const int i32 = (kb - T.kb0) & 31;
+          if (i32 == 0 && kb != T.kb0) {
+            sb_cur = sb_nxt;
+            sb_nxt = kb + 32 + lane < T.kb1 ? __ldg(sbp + kb + 32 + lane) : 0.f;
+          }
+          const float s_b = __shfl_sync(0xffffffffu, sb_cur, i32);
+          // the stage's sa slice is read below: wait for its TMA as well
+          bool w = wait_phase(tfull_bar(b), tph, abort_flag);
+          w = w && wait_phase(full_bar(s), ph, abort_flag);
+          if (!__all_sync(0xffffffffu, w)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                 static_cast<uint32_t>(b * BNC + wg * kCW);
 #pragma unroll
-        for (int j0 = 0; j0 < kChunks; j0 += kGroup) {
-          if (32 * j0 >= live) break;
-          uint32_t r[kGroup][32];
+          for (int j0 = 0; j0 < kChunks; j0 += kGroup) {
+            if (32 * j0 >= live) break;
+            uint32_t r[kGroup][32];
 #pragma unroll
-          for (int j = 0; j < kGroup; ++j)
-            if (32 * (j0 + j) < live) tmem_ld_32x32b_x32(taddr + 32 * (j0 + j), r[j]);
-          tmem_ld_wait_bind(r[0]);
+            for (int j = 0; j < kGroup; ++j)
+              if (32 * (j0 + j) < live) tmem_ld_32x32b_x32(taddr + 32 * (j0 + j), r[j]);
+            tmem_ld_wait_bind(r[0]);
 #pragma unroll
-          for (int j = 1; j < kGroup; ++j) bind_after_wait(r[j]);
+            for (int j = 1; j < kGroup; ++j) bind_after_wait(r[j]);
 #pragma unroll
-          for (int j = 0; j < kGroup; ++j) {
-            if (32 * (j0 + j) >= live) continue;
-            float* a = acc + 32 * (j0 + j);
-            if constexpr (kSwap) {
+            for (int j = 0; j < kGroup; ++j) {
+              if (32 * (j0 + j) >= live) continue;
+              float* a = acc + 32 * (j0 + j);
+              // per column: sa[m0 + c, kb] * sb[nb, kb]
               const float4* f4 = reinterpret_cast<const float4*>(sa_f + s * L::kSaFloats + wg * kCW + 32 * (j0 + j));
 #pragma unroll
               for (int c4 = 0; c4 < 8; ++c4) {
@@ -545,17 +598,14 @@ __global__ void __launch_bounds__(kThreads, MINB)
                 a[4 * c4 + 2] = fmaf(__uint_as_float(r[j][4 * c4 + 2]), f.z * s_b, a[4 * c4 + 2]);
                 a[4 * c4 + 3] = fmaf(__uint_as_float(r[j][4 * c4 + 3]), f.w * s_b, a[4 * c4 + 3]);
               }
-            } else {
-#pragma unroll
-              for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc_row, a[c]);
             }
           }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(tempty_bar(b));
-          mbar_arrive(empty_bar(s));
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(tempty_bar(b));
+            mbar_arrive(empty_bar(s));
+          }
         }
       }
       if (!ok) break;
