@@ -13,6 +13,7 @@
 
 #include "fp8gemm.h"
 #include "kernel.cuh"
+#include "kernel_pair.cuh"
 
 using namespace fp8g;
 
@@ -29,13 +30,20 @@ struct Variant {
   bool reg_split;  // setmaxnreg variant: needs exactly kLaunchRegs at launch
   KernelFn fn;
   int smem;
+  bool pair;  // CTA pairs (clusters of two) sharing a 256 x 256 tile
 };
 
 template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int MINB = 1>
 Variant make_variant(const char* name) {
   using L = Layout<kSwap, BNC, STAGES, SPLIT, MINB>;
   return Variant{name, KIND, kSwap, BNC, STAGES, SPLIT, L::kRegSplit,
-                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT, MINB>, L::kSmemAlloc};
+                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT, MINB>, L::kSmemAlloc, false};
+}
+
+template <int KIND, int STAGES>
+Variant make_pair_variant(const char* name) {
+  return Variant{name, KIND, false, 256, STAGES, 1, true, &fp8_gemm_pair_kernel<KIND, STAGES>,
+                 PairLayout<STAGES>::kSmemAlloc, true};
 }
 
 // "nlanes": TMEM lanes are rows of B (small M); "mlanes": lanes are rows of A.
@@ -57,6 +65,8 @@ const Variant kVariants[] = {
     make_variant<true, 64, 8, kDense, kGlobalSplit>("dense_nlanes_bn64_st8_gsplit"),
     make_variant<true, 64, 8, kDense, kGlobalSplitPartials>("dense_nlanes_bn64_st8_gsplit_2k"),
     make_variant<true, 64, 4, kDense, kGlobalSplitPartials, 2>("dense_nlanes_bn64_st4_gsplit_2k_x2"),
+    make_pair_variant<kDense, 6>("dense_mlanes_pair_bn256_st6"),
+    make_pair_variant<kMasked, 6>("masked_mlanes_pair_bn256_st6"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
@@ -77,6 +87,8 @@ enum : int {
   V_DENSE_GSPLIT = 14,
   V_DENSE_GSPLIT2K = 15,
   V_DENSE_GSPLIT2K_X2 = 16,
+  V_DENSE_PAIR = 17,
+  V_MASKED_PAIR = 18,
 };
 
 std::atomic<int> g_override{-1};
@@ -101,7 +113,7 @@ struct DeviceInfo {
   int sms = 0;
   int max_smem_optin = 0;
   bool attr_set[kNumVariants] = {};
-  int max_clusters[kNumVariants] = {};  // split variants: co-resident clusters
+  int max_clusters[kNumVariants] = {};  // split and pair variants: co-resident clusters
   // global split-K workspace: sms slots of 64 x 128 floats, 2 counters per tile
   float* ws = nullptr;
   uint32_t* sync = nullptr;
@@ -147,17 +159,18 @@ int prepare_variant(DeviceInfo* d, int v) {
   if (cudaFuncSetAttribute(reinterpret_cast<const void*>(V.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
                            V.smem) != cudaSuccess)
     return FP8G_ERR_CUDA;
-  if (V.split > 1) {
+  if (V.split > 1 || V.pair) {
+    const int cs = V.pair ? 2 : V.split;
     if (cudaFuncSetAttribute(reinterpret_cast<const void*>(V.fn), cudaFuncAttributeNonPortableClusterSizeAllowed,
-                             V.split > 8 ? 1 : 0) != cudaSuccess)
+                             cs > 8 ? 1 : 0) != cudaSuccess)
       return FP8G_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = V.split;
+    attr[0].val.clusterDim.x = cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(V.split * 64, 1, 1);
+    cfg.gridDim = dim3(cs * 64, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = V.smem;
     cfg.attrs = attr;
@@ -282,8 +295,10 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   if (rc) return rc;
 
   const int KB = P.K / 128, NB = (P.N + 127) / 128;
-  const int m_ext = V.swap ? V.bnc : 128;
-  const int n_ext = V.swap ? 128 : V.bnc;
+  // output tile: n-lanes BNC rows of A x 128 rows of B; m-lanes 128 x BNC;
+  // pairs 256 x 256 (each CTA loads 128 rows of A and 128 rows of B)
+  const int m_ext = V.pair ? 256 : V.swap ? V.bnc : 128;
+  const int n_ext = V.pair ? 256 : V.swap ? 128 : V.bnc;
   const int G_a = P.kind == kMasked ? P.G : 1;
   const int G_b = P.kind == kDense ? 1 : P.G;
 
@@ -314,7 +329,7 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
 
   CUtensorMap tmA, tmB, tmSA;
   const uint32_t a_box_rows = V.swap ? V.bnc : 128;
-  const uint32_t b_box_rows = V.swap ? 128 : V.bnc;
+  const uint32_t b_box_rows = V.swap || V.pair ? 128 : V.bnc;
   rc = encode3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, P.A, P.K, P.M, G_a, (uint64_t)P.K,
                 (uint64_t)P.K * std::max(P.M, 1), 128, a_box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!rc)
@@ -347,6 +362,15 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
     cfg.gridDim = dim3(p.num_tiles * V.split, 1, 1);
   } else if (V.split < 0) {
     cfg.gridDim = dim3(p.gsplit, p.n_tiles, p.m_tiles);
+  } else if (V.pair) {
+    const int clusters = std::min(p.num_tiles, dev->max_clusters[v]);
+    if (clusters < 1) return FP8G_ERR_UNSUPPORTED;
+    attr[nattr].id = cudaLaunchAttributeClusterDimension;
+    attr[nattr].val.clusterDim.x = 2;
+    attr[nattr].val.clusterDim.y = 1;
+    attr[nattr].val.clusterDim.z = 1;
+    ++nattr;
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
   } else {
     cfg.gridDim = dim3(std::min(p.num_tiles, dev->sms), 1, 1);
   }

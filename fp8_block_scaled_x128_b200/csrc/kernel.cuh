@@ -544,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(b));
+            if (lane == 0) mbar_arrive_relaxed(tempty_bar(b));
             ++it;
           }
         }

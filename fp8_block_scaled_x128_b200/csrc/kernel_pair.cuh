@@ -1,0 +1,321 @@
+// kernel_pair.cuh -- the m-lanes GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+// Same arithmetic as fp8_gemm_kernel with kSwap = false (D rows on TMEM
+// lanes, one scale sa[m,kb] * sb[n/128,kb] per thread and K-block, FP32
+// promotion on the CUDA cores), but a cluster of two CTAs computes a
+// 256 x 256 output tile with one MMA stream:
+//
+//   rank r (0, 1)  holds rows m0 + 128 r .. +127 of A and rows n0 + 128 r ..
+//                  +127 of B for each K-block, in its own shared memory at the
+//                  same offsets as its peer;
+//   rank 0         issues tcgen05.mma.cta_group::2 (M = 256, N = 256), which
+//                  reads both CTAs' operands and writes D rows m0 + 128 r of
+//                  all 256 columns into CTA r's TMEM;
+//   both           promote and store their own 128 rows.
+//
+// Each CTA loads 32 KB per K-block instead of the 48 KB a 128 x 256 tile on
+// one CTA needs, so the pair moves a third less data from L2 per FLOP.
+//
+// Barriers (all in each CTA; the ones marked "rank 0" are used there only):
+//   full[s]    rank 0: both CTAs' TMA bytes of stage s (rank 0 posts the
+//              expected count for both)
+//   empty[s]   stage s consumed: one tcgen05.commit multicast to both CTAs
+//   tfull[b]   partial b ready: one commit multicast to both CTAs
+//   tempty[b]  rank 0: partial b read by the 8 promotion warps of both CTAs
+//              (the peer's arrive remotely)
+// Every wait is bounded as in fp8_gemm_kernel; the CTAs of a pair leave
+// through one cluster barrier after all their work (and aborts) have drained.
+#pragma once
+
+#include "kernel.cuh"
+
+namespace fp8g {
+
+template <int STAGES>
+struct PairLayout {
+  static constexpr int kTileBytes = 128 * 128;  // 128 rows x one K-block of e4m3
+  static constexpr int kNBuf = 2;               // TMEM partial buffers of 256 columns
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = STAGES * kTileBytes;
+  static constexpr int kOffBar = 2 * STAGES * kTileBytes;
+  static constexpr int kNumBars = 2 * STAGES + 2 * kNBuf + 2;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffMisc + 16;
+  static constexpr int kSmemAlloc = kBytes + 1024;
+  static_assert(STAGES % 2 == 0, "stages alternate between the two MMA issuers");
+  static_assert(kSmemAlloc <= 232448, "shared memory");
+};
+
+struct PairTile {
+  int g, m0, n0;  // m0: first row of the pair tile; this CTA's rows start at m0 + 128 * rank
+  int mvalid;     // rows of this CTA's half that exist (may be <= 0)
+  bool valid;     // the pair has work on this tile
+};
+
+template <int KIND>
+__device__ __forceinline__ PairTile get_pair_tile(const Params& p, int t, uint32_t rank, bool report) {
+  PairTile T;
+  T.g = 0;
+  T.valid = true;
+  if constexpr (KIND == kDense) {
+    const int nt = t % p.n_tiles, mt = t / p.n_tiles;
+    T.m0 = mt * 256;
+    T.n0 = nt * 256;
+    T.mvalid = min(128, p.M - (T.m0 + 128 * static_cast<int>(rank)));
+  } else {
+    static_assert(KIND == kMasked, "pair tiles: dense and masked");
+    const int per_g = p.n_tiles * p.m_tiles;
+    const int g = t / per_g, r = t % per_g;
+    const int nt = r / p.m_tiles, mt = r % p.m_tiles;
+    int mg = __ldg(p.masked_m + g);
+    if (mg > p.M) {
+      if (report) atomicOr(&g_fp8g_error_word, FP8G_DEVERR_MASKED_OVER);
+      mg = p.M;
+    }
+    mg = max(mg, 0);
+    T.g = g;
+    T.m0 = mt * 256;
+    T.n0 = nt * 256;
+    T.mvalid = min(128, mg - (T.m0 + 128 * static_cast<int>(rank)));
+    T.valid = T.m0 < mg;
+  }
+  return T;
+}
+
+template <int KIND, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmSA, const Params p) {
+  using L = PairLayout<STAGES>;
+  constexpr int BNC = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+
+  const uint32_t bar0 = sbase + L::kOffBar;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + L::kNBuf + b); };
+  auto drain_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + 2 * L::kNBuf + i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  auto a_tile = [&](int s) { return sbase + L::kOffA + s * L::kTileBytes; };
+  auto b_tile = [&](int s) { return sbase + L::kOffB + s * L::kTileBytes; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < L::kNBuf; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 16);  // every promotion warp of both CTAs
+    }
+    mbar_init(drain_bar(0), 1);
+    mbar_init(drain_bar(1), 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  // the peer's barriers are initialised before either CTA signals the other
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int t_first = static_cast<int>(blockIdx.x / 2);
+  const int t_step = static_cast<int>(gridDim.x / 2);
+
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
+  constexpr uint32_t kPairStageTx = 2u * 2u * L::kTileBytes;  // A and B halves of both CTAs
+
+  if (warp < 4) {
+    setmaxnreg_dec<kControlRegs>();
+    if (warp == 0 || warp == 3) {
+      // ------------------------------------------------------------ producers (both CTAs)
+      if (lane < kIssuersPerWarp) {
+        const uint32_t me = static_cast<uint32_t>((warp == 3 ? kIssuersPerWarp : 0) + lane);
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
+          const PairTile T = get_pair_tile<KIND>(p, t, rank, false);
+          if (!T.valid) continue;
+          const int ga = KIND == kMasked ? T.g : 0;
+          const int gb = KIND == kDense ? 0 : T.g;
+          const int arow = T.m0 + 128 * static_cast<int>(rank);
+          const int brow = T.n0 + 128 * static_cast<int>(rank);
+          for (int kb = 0; kb < p.KB; ++kb, ++it) {
+            if ((it % STAGES) % kIssuers != me) continue;
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1u;
+            if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = rank == 0 ? full_bar(s) : mapa(full_bar(s), 0);
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(s), kPairStageTx);
+            tma_load_3d_pair(a_tile(s), &tmA, fb, kb * 128, arow, ga);
+            tma_load_3d_pair(b_tile(s), &tmB, fb, kb * 128, brow, gb);
+          }
+        }
+        // rank 0 drains: the full barriers count both CTAs' bytes, so every
+        // load of the pair has landed once they complete
+        if (rank == 0) {
+          const uint32_t first = it > static_cast<uint32_t>(STAGES) ? it - STAGES : 0u;
+          for (uint32_t i = first; i < it; ++i)
+            if ((i % STAGES) % kIssuers == me) drain_phase(full_bar(i % STAGES), (i / STAGES) & 1u);
+        }
+      }
+    } else if (rank == 0 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuers (rank 0, warps 1 and 2)
+      const uint32_t me = static_cast<uint32_t>(warp - 1);
+      constexpr uint32_t kIdesc = idesc_e4m3_f32(256, BNC);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
+        const PairTile T = get_pair_tile<KIND>(p, t, rank, false);
+        if (!T.valid) continue;
+        for (int kb = 0; kb < p.KB; ++kb, ++it) {
+          if ((it % STAGES) % 2 != me) continue;
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          const int b = it % L::kNBuf;
+          const uint32_t tph = (it / L::kNBuf) & 1u;
+          if (!wait_phase(full_bar(s), ph, abort_flag) ||
+              !wait_phase(tempty_bar(b), tph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BNC);
+          const uint64_t adesc = sdesc_k128_sw128(a_tile(s));
+          const uint64_t bdesc = sdesc_k128_sw128(b_tile(s));
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_f8f6f4_pair(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k),
+                            kIdesc, k > 0 ? 1u : 0u);
+          mma_commit_pair(empty_bar(s), 0x3);
+          mma_commit_pair(tfull_bar(b), 0x3);
+        }
+      }
+      // drain: every MMA of this thread completes before TMEM is freed
+      mma_commit_pair(drain_bar(me), 0x1);
+      drain_phase(drain_bar(me), 0u);
+    }
+  } else {
+    // ------------------------------------------------------------ promotion + epilogue (both CTAs)
+    setmaxnreg_inc<kPromoRegs>();
+    constexpr int kCW = BNC / 2;  // 128 columns per promotion warpgroup
+    const int wg = (warp - 4) / 4;
+    const int q = warp % 4;
+    const int row = 32 * q + lane;
+    // rank 1 releases TMEM buffers on rank 0's barrier
+    const uint32_t tempty_remote0 = mapa(tempty_bar(0), 0);
+    const uint32_t tempty_remote1 = mapa(tempty_bar(1), 0);
+    float acc[kCW];
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
+      const PairTile T = get_pair_tile<KIND>(p, t, rank, warp == 4 && lane == 0 && rank == 0);
+      if (!T.valid) continue;
+#pragma unroll
+      for (int c = 0; c < kCW; ++c) acc[c] = 0.f;
+      const int m_row = T.m0 + 128 * static_cast<int>(rank) + row;  // this thread's row of A and D
+      const int nb = min((T.n0 + wg * kCW) / 128, p.NB - 1);
+      const float* sbp = p.sb + (static_cast<long>(T.g) * p.NB + nb) * p.KB;
+      const bool row_in = m_row < p.M;
+      const float* sap = p.sa + (KIND == kMasked ? static_cast<long>(T.g) * p.KB * p.ld_sa : 0L) + m_row;
+      auto sa_at = [&](int kb) { return row_in && kb < p.KB ? __ldg(sap + static_cast<long>(kb) * p.ld_sa) : 0.f; };
+      auto sb_at = [&](int kb) { return kb < p.KB ? __ldg(sbp + kb) : 0.f; };
+      float sa0 = sa_at(0), sa1 = sa_at(1);
+      float sb0 = sb_at(0), sb1 = sb_at(1);
+      for (int kb = 0; ok && kb < p.KB; kb += 2) {
+        const float sc2[2] = {sa0 * sb0, sa1 * sb1};
+        sa0 = sa_at(kb + 2);
+        sa1 = sa_at(kb + 3);
+        sb0 = sb_at(kb + 2);
+        sb1 = sb_at(kb + 3);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (kb + u >= p.KB) break;
+          const int b = it % L::kNBuf;
+          const uint32_t tph = (it / L::kNBuf) & 1u;
+          if (!__all_sync(0xffffffffu, wait_phase(tfull_bar(b), tph, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                 static_cast<uint32_t>(b * BNC + wg * kCW);
+#pragma unroll
+          for (int j0 = 0; j0 < kCW / 32; j0 += 2) {
+            uint32_t r[2][32];
+            tmem_ld_32x32b_x32(taddr + 32 * j0, r[0]);
+            tmem_ld_32x32b_x32(taddr + 32 * (j0 + 1), r[1]);
+            tmem_ld_wait_bind(r[0]);
+            bind_after_wait(r[1]);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              float* a = acc + 32 * (j0 + j);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (rank == 0) mbar_arrive_relaxed(tempty_bar(b));
+            else mbar_arrive_remote_relaxed(b == 0 ? tempty_remote0 : tempty_remote1);
+          }
+          ++it;
+        }
+      }
+      if (!ok) break;
+
+      // epilogue: a thread holds 128 consecutive columns of its row
+      if (row < T.mvalid) {
+        const long drow0 = KIND == kMasked ? static_cast<long>(T.g) * p.M : 0;
+        uint16_t* drow = p.D + (drow0 + m_row) * p.N + T.n0 + wg * kCW;
+#pragma unroll
+        for (int c = 0; c < kCW; c += 8) {
+          if (T.n0 + wg * kCW + c < p.N) {
+            uint4 v;
+            v.x = pack_bf16x2(acc[c + 0], acc[c + 1]);
+            v.y = pack_bf16x2(acc[c + 2], acc[c + 3]);
+            v.z = pack_bf16x2(acc[c + 4], acc[c + 5]);
+            v.w = pack_bf16x2(acc[c + 6], acc[c + 7]);
+            *reinterpret_cast<uint4*>(drow + c) = v;
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  // rank 0's MMAs into rank 1's TMEM, rank 1's loads counted on rank 0's
+  // barriers and rank 1's remote arrivals are all finished past this point
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
+}  // namespace fp8g
