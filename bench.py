@@ -105,6 +105,12 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def kernels_per_call(variant: str) -> int:
+    """Kernels one C-ABI call launches: the two-kernel split-K variants run a
+    partial-sums kernel and a reduce kernel, all others one kernel."""
+    return 2 if "gsplit_2k" in variant else 1
+
+
 def ncu_traffic(workload: str, variant: str):
     """DRAM bytes per launch from the committed ncu summary of this kernel and
     workload, if it was taken on the current kernel sources (else None)."""
@@ -439,6 +445,8 @@ def run_ours(args, rank: int, world: int) -> None:
     roof["avg_launch_us"] = avg_launch_s * 1e6
     roof["launch_time_source"] = ("CUDA events around every launch" if args.per_launch_events else
                                   "CUDA events around the K back-to-back launches of the timed region, / K")
+    if kernels_per_call(variant) > 1:
+        roof["launch_time_source"] += " (a call is the partial-sums kernel and its reduce kernel)"
 
     value = world * acc["flops"] * args.steps / (ms_max * 1e-3) / 1e12
     line = {
@@ -452,7 +460,8 @@ def run_ours(args, rank: int, world: int) -> None:
                           if copies > 1 else f"inputs {per_copy / 2**20:.0f} MiB >= 2x L2"),
                    "launch": "CUDA graph of the K steps, one C-ABI call each",
                    "variant": variant, "parallelism": "replicas" if world > 1 else "single GPU"},
-        "roofline": roof, "gpu_launches": world * args.steps, "clocks": clocks, "e2e": e2e,
+        "roofline": roof, "gpu_launches": world * args.steps * kernels_per_call(variant), "clocks": clocks,
+        "e2e": e2e,
     }
     if remeasured:
         line["clocks_remeasured"] = True
