@@ -27,23 +27,26 @@ struct Variant {
   int kind;
   bool swap;
   int bnc, stages, split;
-  bool reg_split;  // setmaxnreg variant: needs exactly kLaunchRegs at launch
+  bool reg_split;  // setmaxnreg variant: needs exactly launch_regs at launch
   KernelFn fn;
   int smem;
-  bool pair;  // CTA pairs (clusters of two) sharing a 256 x 256 tile
+  bool pair;        // CTA pairs (clusters of two) sharing a 256 x bnc tile
+  int threads;      // threads per CTA
+  int launch_regs;  // register-split variants: registers per thread at launch
 };
 
-template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int MINB = 1>
+template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int MINB = 1, bool HALF = false>
 Variant make_variant(const char* name) {
-  using L = Layout<kSwap, BNC, STAGES, SPLIT, MINB>;
+  using L = Layout<kSwap, BNC, STAGES, SPLIT, MINB, HALF>;
   return Variant{name, KIND, kSwap, BNC, STAGES, SPLIT, L::kRegSplit,
-                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT, MINB>, L::kSmemAlloc, false};
+                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT, MINB, HALF>, L::kSmemAlloc, false,
+                 kThreads, kLaunchRegs};
 }
 
-template <int KIND, int STAGES>
+template <int KIND, int STAGES, int BN>
 Variant make_pair_variant(const char* name) {
-  return Variant{name, KIND, false, 256, STAGES, 1, true, &fp8_gemm_pair_kernel<KIND, STAGES>,
-                 PairLayout<STAGES>::kSmemAlloc, true};
+  return Variant{name, KIND, false, BN, STAGES, 1, true, &fp8_gemm_pair_kernel<KIND, STAGES, BN>,
+                 PairLayout<STAGES, BN>::kSmemAlloc, true, PairShape<BN>::kThreads, PairShape<BN>::kLaunchRegs};
 }
 
 // "nlanes": TMEM lanes are rows of B (small M); "mlanes": lanes are rows of A.
@@ -65,8 +68,14 @@ const Variant kVariants[] = {
     make_variant<true, 64, 8, kDense, kGlobalSplit>("dense_nlanes_bn64_st8_gsplit"),
     make_variant<true, 64, 8, kDense, kGlobalSplitPartials>("dense_nlanes_bn64_st8_gsplit_2k"),
     make_variant<true, 64, 4, kDense, kGlobalSplitPartials, 2>("dense_nlanes_bn64_st4_gsplit_2k_x2"),
-    make_pair_variant<kDense, 6>("dense_mlanes_pair_bn256_st6"),
-    make_pair_variant<kMasked, 6>("masked_mlanes_pair_bn256_st6"),
+    make_pair_variant<kDense, 6, 256>("dense_mlanes_pair_bn256_st6"),
+    make_pair_variant<kMasked, 6, 256>("masked_mlanes_pair_bn256_st6"),
+    make_variant<false, 256, 4, kDense, 1, 1, true>("dense_mlanes_bn256h_st4"),
+    make_variant<false, 256, 4, kContiguous, 1, 1, true>("contiguous_mlanes_bn256h_st4"),
+    make_variant<false, 256, 4, kMasked, 1, 1, true>("masked_mlanes_bn256h_st4"),
+    make_pair_variant<kDense, 6, 192>("dense_mlanes_pair_bn192_st6"),
+    make_pair_variant<kMasked, 6, 192>("masked_mlanes_pair_bn192_st6"),
+    make_pair_variant<kContiguous, 6, 192>("contiguous_mlanes_pair_bn192_st6"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
@@ -89,6 +98,12 @@ enum : int {
   V_DENSE_GSPLIT2K_X2 = 16,
   V_DENSE_PAIR = 17,
   V_MASKED_PAIR = 18,
+  V_DENSE_M256H = 19,
+  V_CONTIG_M256H = 20,
+  V_MASKED_M256H = 21,
+  V_DENSE_PAIR192 = 22,
+  V_MASKED_PAIR192 = 23,
+  V_CONTIG_PAIR192 = 24,
 };
 
 std::atomic<int> g_override{-1};
@@ -150,11 +165,11 @@ int prepare_variant(DeviceInfo* d, int v) {
   const Variant& V = kVariants[v];
   if (V.smem > d->max_smem_optin) return FP8G_ERR_UNSUPPORTED;
   if (V.reg_split) {
-    // the setmaxnreg split is sized for exactly kLaunchRegs per thread at
+    // the setmaxnreg split is sized for exactly launch_regs per thread at
     // launch; any other count would leave the promotion warps waiting
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(V.fn)) != cudaSuccess) return FP8G_ERR_CUDA;
-    if (fa.numRegs != kLaunchRegs) return FP8G_ERR_UNSUPPORTED;
+    if (fa.numRegs != V.launch_regs) return FP8G_ERR_UNSUPPORTED;
   }
   if (cudaFuncSetAttribute(reinterpret_cast<const void*>(V.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
                            V.smem) != cudaSuccess)
@@ -171,7 +186,7 @@ int prepare_variant(DeviceInfo* d, int v) {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(cs * 64, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(V.threads, 1, 1);
     cfg.dynamicSmemBytes = V.smem;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -298,7 +313,7 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   // output tile: n-lanes BNC rows of A x 128 rows of B; m-lanes 128 x BNC;
   // pairs 256 x 256 (each CTA loads 128 rows of A and 128 rows of B)
   const int m_ext = V.pair ? 256 : V.swap ? V.bnc : 128;
-  const int n_ext = V.pair ? 256 : V.swap ? 128 : V.bnc;
+  const int n_ext = V.pair ? V.bnc : V.swap ? 128 : V.bnc;
   const int G_a = P.kind == kMasked ? P.G : 1;
   const int G_b = P.kind == kDense ? 1 : P.G;
 
@@ -310,7 +325,8 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   p.NB = NB;
   p.G = G_b;
   p.n_tiles = (P.N + n_ext - 1) / n_ext;
-  p.m_tiles = P.kind == kContiguous ? P.M / 128 : (P.M + m_ext - 1) / m_ext;
+  // contiguous: 128-row expert blocks, two per pair tile
+  p.m_tiles = P.kind != kContiguous ? (P.M + m_ext - 1) / m_ext : V.pair ? (P.M / 128 + 1) / 2 : P.M / 128;
   p.num_tiles = p.n_tiles * p.m_tiles * (P.kind == kMasked ? P.G : 1);
   p.m_indices = P.kind == kContiguous ? P.idx : nullptr;
   p.masked_m = P.kind == kMasked ? P.idx : nullptr;
@@ -329,7 +345,7 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
 
   CUtensorMap tmA, tmB, tmSA;
   const uint32_t a_box_rows = V.swap ? V.bnc : 128;
-  const uint32_t b_box_rows = V.swap || V.pair ? 128 : V.bnc;
+  const uint32_t b_box_rows = V.pair ? V.bnc / 2 : V.swap ? 128 : V.bnc;
   rc = encode3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, P.A, P.K, P.M, G_a, (uint64_t)P.K,
                 (uint64_t)P.K * std::max(P.M, 1), 128, a_box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!rc)
@@ -343,7 +359,7 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   unsigned nattr = 0;
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(V.threads, 1, 1);
   cfg.dynamicSmemBytes = V.smem;
   cfg.stream = stream;
   if (pdl_enabled()) {
@@ -411,12 +427,23 @@ int select_variant(const Problem& P, DeviceInfo* dev, cudaStream_t stream) {
   auto wide = [&](int v256, int v128, long tiles256) {
     return tiles256 >= dev->sms && prepare_variant(dev, v256) == FP8G_OK ? v256 : v128;
   };
+  // CTA pairs, 256 x 192 tiles, when there are enough to give every
+  // co-resident cluster one
+  auto pair = [&](int v, long pair_tiles) {
+    return prepare_variant(dev, v) == FP8G_OK && dev->max_clusters[v] > 0 && pair_tiles >= dev->max_clusters[v];
+  };
+  // contiguous: the pair variant is correct for any expert layout (a pair
+  // tile that straddles two experts runs once per expert) but measured
+  // slower than the single-CTA tiles on G=4, M=8192 per expert, N=4096,
+  // K=7168 (1295 vs 1257 us), so it is only reached by an explicit choice
   if (P.kind == kContiguous)
     return wide(V_CONTIG_M256, V_CONTIG_M128, static_cast<long>(P.M / 128) * ((P.N + 255) / 256));
   if (P.kind == kMasked) {
-    if (P.expected_m > 0 && P.expected_m <= 64) return V_MASKED_N64;
-    // B streams once per 128 rows of a group's A: m-lanes tiles read it the
-    // fewest times; count the tiles the typical group fills
+    // B streams once per 128 (or 256) rows of a group's A: m-lanes tiles read
+    // it the fewest times; count the tiles the typical group fills
+    if (P.expected_m > 0 && P.expected_m <= 64) return V_MASKED_M128;
+    const long m_pairs = (std::max(P.expected_m, 1) + 255) / 256;
+    if (pair(V_MASKED_PAIR192, static_cast<long>(P.G) * m_pairs * ((P.N + 191) / 192))) return V_MASKED_PAIR192;
     const long m_blocks = (std::max(P.expected_m, 1) + 127) / 128;
     return wide(V_MASKED_M256, V_MASKED_M128, static_cast<long>(P.G) * m_blocks * ((P.N + 255) / 256));
   }
@@ -437,6 +464,7 @@ int select_variant(const Problem& P, DeviceInfo* dev, cudaStream_t stream) {
     }
     return V_DENSE_N64;
   }
+  if (pair(V_DENSE_PAIR192, static_cast<long>((P.M + 255) / 256) * ((P.N + 191) / 192))) return V_DENSE_PAIR192;
   return wide(V_DENSE_M256, V_DENSE_M128, static_cast<long>((P.M + 127) / 128) * ((P.N + 255) / 256));
 }
 

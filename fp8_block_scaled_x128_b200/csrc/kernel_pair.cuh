@@ -3,18 +3,18 @@
 // Same arithmetic as fp8_gemm_kernel with kSwap = false (D rows on TMEM
 // lanes, one scale sa[m,kb] * sb[n/128,kb] per thread and K-block, FP32
 // promotion on the CUDA cores), but a cluster of two CTAs computes a
-// 256 x 256 output tile with one MMA stream:
+// 256 x BN output tile (BN = 256 or 192) with one MMA stream:
 //
-//   rank r (0, 1)  holds rows m0 + 128 r .. +127 of A and rows n0 + 128 r ..
-//                  +127 of B for each K-block, in its own shared memory at the
+//   rank r (0, 1)  holds rows m0 + 128 r .. +127 of A and rows n0 + BN/2 r ..
+//                  + BN/2 - 1 of B for each K-block, in its own shared memory at the
 //                  same offsets as its peer;
-//   rank 0         issues tcgen05.mma.cta_group::2 (M = 256, N = 256), which
+//   rank 0         issues tcgen05.mma.cta_group::2 (M = 256, N = BN), which
 //                  reads both CTAs' operands and writes D rows m0 + 128 r of
-//                  all 256 columns into CTA r's TMEM;
+//                  all BN columns into CTA r's TMEM;
 //   both           promote and store their own 128 rows.
 //
-// Each CTA loads 32 KB per K-block instead of the 48 KB a 128 x 256 tile on
-// one CTA needs, so the pair moves a third less data from L2 per FLOP.
+// With BN = 256 each CTA loads 32 KB per K-block instead of the 48 KB a 128 x
+// 256 tile on one CTA needs: a third less data from L2 per FLOP.
 //
 // Barriers (all in each CTA; the ones marked "rank 0" are used there only):
 //   full[s]    rank 0: both CTAs' TMA bytes of stage s (rank 0 posts the
@@ -31,39 +31,93 @@
 
 namespace fp8g {
 
-template <int STAGES>
+// BN: columns of the pair tile (the MMA's N).  256: two promotion
+// warpgroups of 128 columns; 192: three of 64 columns (512 threads), which
+// spreads the FP32 promotion over more warps at the cost of a narrower tile.
+template <int BN>
+struct PairShape {
+  static_assert(BN == 256 || BN == 192, "pair tile width");
+  static constexpr int kNWG = BN == 192 ? 3 : 2;          // promotion warpgroups
+  static constexpr int kCW = BN / kNWG;                   // columns per promotion thread
+  static constexpr int kThreads = 128 * (1 + kNWG);
+  static constexpr int kLaunchRegs = kNWG == 2 ? 168 : 128;
+  static constexpr int kControlRegs = 56;
+  static constexpr int kPromoRegs = kNWG == 2 ? 224 : 152;
+  static constexpr int kGroup = kCW >= 128 ? 2 : 1;       // 32-column TMEM loads per wait
+  static_assert(128 * kControlRegs + 128 * kNWG * kPromoRegs <= kThreads * kLaunchRegs, "register split");
+  static_assert(kThreads * kLaunchRegs <= 65536, "register file");
+};
+
+template <int STAGES, int BN = 256>
 struct PairLayout {
-  static constexpr int kTileBytes = 128 * 128;  // 128 rows x one K-block of e4m3
-  static constexpr int kNBuf = 2;               // TMEM partial buffers of 256 columns
+  static constexpr int kTileBytes = 128 * 128;       // A: 128 rows x one K-block of e4m3
+  static constexpr int kBTileBytes = (BN / 2) * 128;  // B: this CTA's BN / 2 rows
+  static constexpr int kNBuf = 2;                     // TMEM partial buffers of BN columns
   static constexpr int kOffA = 0;
   static constexpr int kOffB = STAGES * kTileBytes;
-  static constexpr int kOffBar = 2 * STAGES * kTileBytes;
+  static constexpr int kOffBar = kOffB + STAGES * kBTileBytes;
   static constexpr int kNumBars = 2 * STAGES + 2 * kNBuf + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;
   static_assert(STAGES % 2 == 0, "stages alternate between the two MMA issuers");
+  static_assert(kBTileBytes % 1024 == 0, "swizzle-128B tiles need 1024 alignment");
   static_assert(kSmemAlloc <= 232448, "shared memory");
 };
 
 struct PairTile {
-  int g, m0, n0;  // m0: first row of the pair tile; this CTA's rows start at m0 + 128 * rank
-  int mvalid;     // rows of this CTA's half that exist (may be <= 0)
-  bool valid;     // the pair has work on this tile
+  int g, m0, n0;  // g: group of B (and of A, masked); m0: first row of the pair tile, this CTA's rows start at m0 + 128 * rank
+  int mvalid;     // rows of this CTA's half to store (may be <= 0)
+  bool valid;     // the pair has work on this (tile, pass)
+  bool active;    // this CTA accumulates and stores in this pass
 };
 
-template <int KIND>
-__device__ __forceinline__ PairTile get_pair_tile(const Params& p, int t, uint32_t rank, bool report) {
+// Tile t, pass ps -> work of this CTA.  Dense and masked tiles have one
+// pass.  A contiguous pair tile covers two 128-row blocks of A; when they
+// belong to one expert it has one pass, otherwise one pass per expert block
+// (the MMA runs over the whole pair each time and only the CTA whose block
+// belongs to that expert keeps the result).  Every role calls this with the
+// same (t, ps) and gets the same answer.
+template <int KIND, int BN>
+__device__ __forceinline__ PairTile get_pair_tile(const Params& p, int t, int ps, uint32_t rank, bool report) {
   PairTile T;
   T.g = 0;
-  T.valid = true;
-  if constexpr (KIND == kDense) {
+  T.valid = ps == 0;
+  T.active = true;
+  if constexpr (KIND == kContiguous) {
+    const int nt = t % p.n_tiles, mt = t / p.n_tiles;
+    const int mb = p.M / 128;  // 128-row blocks of A
+    int e[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int blk = 2 * mt + h;
+      e[h] = blk < mb ? __ldg(p.m_indices + blk) : -1;
+      if (e[h] >= p.G) {
+        if (report && ps == 0) atomicOr(&g_fp8g_error_word, FP8G_DEVERR_BAD_M_INDEX);
+        e[h] = -1;
+      }
+    }
+    T.m0 = mt * 256;
+    T.n0 = nt * BN;
+    if (e[0] == e[1]) {
+      T.valid = ps == 0 && e[0] >= 0;
+      T.g = e[0];
+    } else {
+      // passes: block 0's expert (if any), then block 1's (if any)
+      const int first = e[0] >= 0 ? 0 : 1;
+      const int owner = ps == 0 ? first : 1;
+      T.valid = (ps == 0 && e[first] >= 0) || (ps == 1 && first == 0 && e[1] >= 0);
+      T.g = e[owner];
+      T.active = static_cast<uint32_t>(owner) == rank;
+    }
+    T.mvalid = T.active ? min(128, p.M - (T.m0 + 128 * static_cast<int>(rank))) : 0;
+  } else if constexpr (KIND == kDense) {
     const int nt = t % p.n_tiles, mt = t / p.n_tiles;
     T.m0 = mt * 256;
-    T.n0 = nt * 256;
+    T.n0 = nt * BN;
     T.mvalid = min(128, p.M - (T.m0 + 128 * static_cast<int>(rank)));
   } else {
-    static_assert(KIND == kMasked, "pair tiles: dense and masked");
+    static_assert(KIND == kMasked, "pair tiles: dense, contiguous and masked");
     const int per_g = p.n_tiles * p.m_tiles;
     const int g = t / per_g, r = t % per_g;
     const int nt = r / p.m_tiles, mt = r % p.m_tiles;
@@ -75,19 +129,20 @@ __device__ __forceinline__ PairTile get_pair_tile(const Params& p, int t, uint32
     mg = max(mg, 0);
     T.g = g;
     T.m0 = mt * 256;
-    T.n0 = nt * 256;
+    T.n0 = nt * BN;
     T.mvalid = min(128, mg - (T.m0 + 128 * static_cast<int>(rank)));
-    T.valid = T.m0 < mg;
+    T.valid = ps == 0 && T.m0 < mg;
   }
   return T;
 }
 
-template <int KIND, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int KIND, int STAGES, int BN = 256>
+__global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmSA, const Params p) {
-  using L = PairLayout<STAGES>;
-  constexpr int BNC = 256;
+  using L = PairLayout<STAGES, BN>;
+  using S = PairShape<BN>;
+  constexpr int BNC = BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -105,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   auto a_tile = [&](int s) { return sbase + L::kOffA + s * L::kTileBytes; };
-  auto b_tile = [&](int s) { return sbase + L::kOffB + s * L::kTileBytes; };
+  auto b_tile = [&](int s) { return sbase + L::kOffB + s * L::kBTileBytes; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -114,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < L::kNBuf; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 16);  // every promotion warp of both CTAs
+      mbar_init(tempty_bar(b), 2 * 4 * S::kNWG);  // every promotion warp of both CTAs
     }
     mbar_init(drain_bar(0), 1);
     mbar_init(drain_bar(1), 1);
@@ -141,23 +196,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   grid_dependency_wait();
   if (threadIdx.x == 0) grid_launch_dependents();
-  constexpr uint32_t kPairStageTx = 2u * 2u * L::kTileBytes;  // A and B halves of both CTAs
+  constexpr uint32_t kPairStageTx = 2u * (L::kTileBytes + L::kBTileBytes);  // A and B parts of both CTAs
+  constexpr int kPasses = KIND == kContiguous ? 2 : 1;
 
   if (warp < 4) {
-    setmaxnreg_dec<kControlRegs>();
+    setmaxnreg_dec<S::kControlRegs>();
     if (warp == 0 || warp == 3) {
       // ------------------------------------------------------------ producers (both CTAs)
       if (lane < kIssuersPerWarp) {
         const uint32_t me = static_cast<uint32_t>((warp == 3 ? kIssuersPerWarp : 0) + lane);
         uint32_t it = 0;
         bool ok = true;
-        for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
-          const PairTile T = get_pair_tile<KIND>(p, t, rank, false);
+        for (int t = t_first; ok && t < p.num_tiles; t += t_step)
+        for (int ps = 0; ok && ps < kPasses; ++ps) {
+          const PairTile T = get_pair_tile<KIND, BN>(p, t, ps, rank, false);
           if (!T.valid) continue;
           const int ga = KIND == kMasked ? T.g : 0;
           const int gb = KIND == kDense ? 0 : T.g;
           const int arow = T.m0 + 128 * static_cast<int>(rank);
-          const int brow = T.n0 + 128 * static_cast<int>(rank);
+          const int brow = T.n0 + (BN / 2) * static_cast<int>(rank);
           for (int kb = 0; kb < p.KB; ++kb, ++it) {
             if ((it % STAGES) % kIssuers != me) continue;
             const int s = it % STAGES;
@@ -186,8 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kIdesc = idesc_e4m3_f32(256, BNC);
       uint32_t it = 0;
       bool ok = true;
-      for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
-        const PairTile T = get_pair_tile<KIND>(p, t, rank, false);
+      for (int t = t_first; ok && t < p.num_tiles; t += t_step)
+      for (int ps = 0; ok && ps < kPasses; ++ps) {
+        const PairTile T = get_pair_tile<KIND, BN>(p, t, ps, rank, false);
         if (!T.valid) continue;
         for (int kb = 0; kb < p.KB; ++kb, ++it) {
           if ((it % STAGES) % 2 != me) continue;
@@ -218,8 +276,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ promotion + epilogue (both CTAs)
-    setmaxnreg_inc<kPromoRegs>();
-    constexpr int kCW = BNC / 2;  // 128 columns per promotion warpgroup
+    setmaxnreg_inc<S::kPromoRegs>();
+    constexpr int kCW = S::kCW;  // columns per promotion warpgroup
     const int wg = (warp - 4) / 4;
     const int q = warp % 4;
     const int row = 32 * q + lane;
@@ -229,8 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float acc[kCW];
     uint32_t it = 0;
     bool ok = true;
-    for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
-      const PairTile T = get_pair_tile<KIND>(p, t, rank, warp == 4 && lane == 0 && rank == 0);
+    for (int t = t_first; ok && t < p.num_tiles; t += t_step)
+    for (int ps = 0; ok && ps < kPasses; ++ps) {
+      const PairTile T = get_pair_tile<KIND, BN>(p, t, ps, rank, warp == 4 && lane == 0 && rank == 0);
       if (!T.valid) continue;
 #pragma unroll
       for (int c = 0; c < kCW; ++c) acc[c] = 0.f;
@@ -261,18 +320,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
                                  static_cast<uint32_t>(b * BNC + wg * kCW);
+          constexpr int kG = S::kGroup;
+          // a CTA whose block belongs to the other expert of this pass only
+          // hands the buffer back
+          if (T.active) {
 #pragma unroll
-          for (int j0 = 0; j0 < kCW / 32; j0 += 2) {
-            uint32_t r[2][32];
-            tmem_ld_32x32b_x32(taddr + 32 * j0, r[0]);
-            tmem_ld_32x32b_x32(taddr + 32 * (j0 + 1), r[1]);
-            tmem_ld_wait_bind(r[0]);
-            bind_after_wait(r[1]);
+            for (int j0 = 0; j0 < kCW / 32; j0 += kG) {
+              uint32_t r[kG][32];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              float* a = acc + 32 * (j0 + j);
+              for (int j = 0; j < kG; ++j) tmem_ld_32x32b_x32(taddr + 32 * (j0 + j), r[j]);
+              tmem_ld_wait_bind(r[0]);
 #pragma unroll
-              for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
+              for (int j = 1; j < kG; ++j) bind_after_wait(r[j]);
+#pragma unroll
+              for (int j = 0; j < kG; ++j) {
+                float* a = acc + 32 * (j0 + j);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
+              }
             }
           }
           tc_fence_before();
@@ -286,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
 
-      // epilogue: a thread holds 128 consecutive columns of its row
+      // epilogue: a thread holds kCW consecutive columns of its row
       if (row < T.mvalid) {
         const long drow0 = KIND == kMasked ? static_cast<long>(T.g) * p.M : 0;
         uint16_t* drow = p.D + (drow0 + m_row) * p.N + T.n0 + wg * kCW;
