@@ -45,7 +45,7 @@ Variant make_variant(const char* name) {
 
 template <int KIND, int STAGES, int BN>
 Variant make_pair_variant(const char* name) {
-  return Variant{name, KIND, false, BN, STAGES, 1, true, &fp8_gemm_pair_kernel<KIND, STAGES, BN>,
+  return Variant{name, KIND, false, BN, STAGES, 1, PairShape<BN>::kRegSplit, &fp8_gemm_pair_kernel<KIND, STAGES, BN>,
                  PairLayout<STAGES, BN>::kSmemAlloc, true, PairShape<BN>::kThreads, PairShape<BN>::kLaunchRegs};
 }
 
@@ -76,6 +76,9 @@ const Variant kVariants[] = {
     make_pair_variant<kDense, 6, 192>("dense_mlanes_pair_bn192_st6"),
     make_pair_variant<kMasked, 6, 192>("masked_mlanes_pair_bn192_st6"),
     make_pair_variant<kContiguous, 6, 192>("contiguous_mlanes_pair_bn192_st6"),
+    make_pair_variant<kDense, 8, 128>("dense_mlanes_pair_bn128_st8"),
+    make_pair_variant<kContiguous, 8, 128>("contiguous_mlanes_pair_bn128_st8"),
+    make_pair_variant<kMasked, 8, 128>("masked_mlanes_pair_bn128_st8"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
@@ -104,6 +107,9 @@ enum : int {
   V_DENSE_PAIR192 = 22,
   V_MASKED_PAIR192 = 23,
   V_CONTIG_PAIR192 = 24,
+  V_DENSE_PAIR128 = 25,
+  V_CONTIG_PAIR128 = 26,
+  V_MASKED_PAIR128 = 27,
 };
 
 std::atomic<int> g_override{-1};

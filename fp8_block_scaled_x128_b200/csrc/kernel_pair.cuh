@@ -33,14 +33,17 @@ namespace fp8g {
 
 // BN: columns of the pair tile (the MMA's N).  256: two promotion
 // warpgroups of 128 columns; 192: three of 64 columns (512 threads), which
-// spreads the FP32 promotion over more warps at the cost of a narrower tile.
+// spreads the FP32 promotion over more warps at the cost of a narrower tile;
+// 128: two of 64 columns and four TMEM buffers instead of two, so the MMA may
+// run up to three K-blocks ahead of the promotion.
 template <int BN>
 struct PairShape {
-  static_assert(BN == 256 || BN == 192, "pair tile width");
+  static_assert(BN == 256 || BN == 192 || BN == 128, "pair tile width");
   static constexpr int kNWG = BN == 192 ? 3 : 2;          // promotion warpgroups
   static constexpr int kCW = BN / kNWG;                   // columns per promotion thread
   static constexpr int kThreads = 128 * (1 + kNWG);
   static constexpr int kLaunchRegs = kNWG == 2 ? 168 : 128;
+  static constexpr bool kRegSplit = kCW > 64 || kNWG == 3;  // setmaxnreg between the roles
   static constexpr int kControlRegs = 56;
   static constexpr int kPromoRegs = kNWG == 2 ? 224 : 152;
   static constexpr int kGroup = kCW >= 128 ? 2 : 1;       // 32-column TMEM loads per wait
@@ -52,7 +55,7 @@ template <int STAGES, int BN = 256>
 struct PairLayout {
   static constexpr int kTileBytes = 128 * 128;       // A: 128 rows x one K-block of e4m3
   static constexpr int kBTileBytes = (BN / 2) * 128;  // B: this CTA's BN / 2 rows
-  static constexpr int kNBuf = 2;                     // TMEM partial buffers of BN columns
+  static constexpr int kNBuf = 512 / BN >= 4 ? 4 : 2;  // TMEM partial buffers of BN columns
   static constexpr int kOffA = 0;
   static constexpr int kOffB = STAGES * kTileBytes;
   static constexpr int kOffBar = kOffB + STAGES * kBTileBytes;
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
   constexpr int kPasses = KIND == kContiguous ? 2 : 1;
 
   if (warp < 4) {
-    setmaxnreg_dec<S::kControlRegs>();
+    if constexpr (S::kRegSplit) setmaxnreg_dec<S::kControlRegs>();
     if (warp == 0 || warp == 3) {
       // ------------------------------------------------------------ producers (both CTAs)
       if (lane < kIssuersPerWarp) {
@@ -276,14 +279,14 @@ __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ promotion + epilogue (both CTAs)
-    setmaxnreg_inc<S::kPromoRegs>();
+    if constexpr (S::kRegSplit) setmaxnreg_inc<S::kPromoRegs>();
+    // rank 1 releases TMEM buffers on rank 0's barriers (consecutive offsets
+    // in rank 0's shared memory window)
+    const uint32_t tempty_remote = mapa(tempty_bar(0), 0);
     constexpr int kCW = S::kCW;  // columns per promotion warpgroup
     const int wg = (warp - 4) / 4;
     const int q = warp % 4;
     const int row = 32 * q + lane;
-    // rank 1 releases TMEM buffers on rank 0's barrier
-    const uint32_t tempty_remote0 = mapa(tempty_bar(0), 0);
-    const uint32_t tempty_remote1 = mapa(tempty_bar(1), 0);
     float acc[kCW];
     uint32_t it = 0;
     bool ok = true;
@@ -344,7 +347,7 @@ __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
           __syncwarp();
           if (lane == 0) {
             if (rank == 0) mbar_arrive_relaxed(tempty_bar(b));
-            else mbar_arrive_remote_relaxed(b == 0 ? tempty_remote0 : tempty_remote1);
+            else mbar_arrive_remote_relaxed(tempty_remote + 8u * b);
           }
           ++it;
         }
