@@ -79,6 +79,8 @@ const Variant kVariants[] = {
     make_pair_variant<kDense, 8, 128>("dense_mlanes_pair_bn128_st8"),
     make_pair_variant<kContiguous, 8, 128>("contiguous_mlanes_pair_bn128_st8"),
     make_pair_variant<kMasked, 8, 128>("masked_mlanes_pair_bn128_st8"),
+    make_pair_variant<kDense, 8, 192>("dense_mlanes_pair_bn192_st8"),
+    make_pair_variant<kMasked, 8, 192>("masked_mlanes_pair_bn192_st8"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
@@ -110,6 +112,8 @@ enum : int {
   V_DENSE_PAIR128 = 25,
   V_CONTIG_PAIR128 = 26,
   V_MASKED_PAIR128 = 27,
+  V_DENSE_PAIR192_S8 = 28,
+  V_MASKED_PAIR192_S8 = 29,
 };
 
 std::atomic<int> g_override{-1};
@@ -470,7 +474,7 @@ int select_variant(const Problem& P, DeviceInfo* dev, cudaStream_t stream) {
     }
     return V_DENSE_N64;
   }
-  if (pair(V_DENSE_PAIR192, static_cast<long>((P.M + 255) / 256) * ((P.N + 191) / 192))) return V_DENSE_PAIR192;
+  if (pair(V_DENSE_PAIR192_S8, static_cast<long>((P.M + 255) / 256) * ((P.N + 191) / 192))) return V_DENSE_PAIR192_S8;
   return wide(V_DENSE_M256, V_DENSE_M128, static_cast<long>((P.M + 127) / 128) * ((P.N + 255) / 256));
 }
 

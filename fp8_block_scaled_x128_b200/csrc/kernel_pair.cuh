@@ -115,7 +115,13 @@ __device__ __forceinline__ PairTile get_pair_tile(const Params& p, int t, int ps
     }
     T.mvalid = T.active ? min(128, p.M - (T.m0 + 128 * static_cast<int>(rank))) : 0;
   } else if constexpr (KIND == kDense) {
-    const int nt = t % p.n_tiles, mt = t / p.n_tiles;
+    // grouped raster: runs of kGroupM pair rows, N fastest within a run's
+    // columns, so that the tiles in flight share few A and B tiles in L2
+    constexpr int kGroupM = 8;
+    const int per_group = kGroupM * p.n_tiles;
+    const int grp = t / per_group, r = t % per_group;
+    const int gm = min(kGroupM, p.m_tiles - grp * kGroupM);
+    const int mt = grp * kGroupM + r % gm, nt = r / gm;
     T.m0 = mt * 256;
     T.n0 = nt * BN;
     T.mvalid = min(128, p.M - (T.m0 + 128 * static_cast<int>(rank)));
