@@ -451,9 +451,11 @@ int select_variant(const Problem& P, DeviceInfo* dev, cudaStream_t stream) {
   if (P.kind == kMasked) {
     // B streams once per 128 (or 256) rows of a group's A: m-lanes tiles read
     // it the fewest times; count the tiles the typical group fills
-    if (P.expected_m > 0 && P.expected_m <= 64) return V_MASKED_M128;
+    // (G=16, N=4096, K=7168, masked_m <= 64: pair 140 us, m-lanes 128 148 us,
+    // n-lanes 64 254 us)
     const long m_pairs = (std::max(P.expected_m, 1) + 255) / 256;
     if (pair(V_MASKED_PAIR192, static_cast<long>(P.G) * m_pairs * ((P.N + 191) / 192))) return V_MASKED_PAIR192;
+    if (P.expected_m > 0 && P.expected_m <= 64) return V_MASKED_M128;
     const long m_blocks = (std::max(P.expected_m, 1) + 127) / 128;
     return wide(V_MASKED_M256, V_MASKED_M128, static_cast<long>(P.G) * m_blocks * ((P.N + 255) / 256));
   }
