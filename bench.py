@@ -105,6 +105,24 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of the ranks' values (every rank gets it): a multi-GPU time
+    is the slowest replica's, never the wall clock of one of them."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_step: float, steps: int, ms: float) -> float:
+    """Aggregate throughput of `world` replicas that each ran `steps` steps in
+    at most `ms` milliseconds."""
+    return world * flops_per_step * steps / (ms * 1e-3) / 1e12
+
+
 def kernels_per_call(variant: str) -> int:
     """Kernels one C-ABI call launches: the two-kernel split-K variants run a
     partial-sums kernel and a reduce kernel, all others one kernel."""
@@ -379,11 +397,7 @@ def run_ours(args, rank: int, world: int) -> None:
     if err:
         raise RuntimeError(f"device error word {err:#x} after the timed region")
 
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
 
     # end to end through the public API: pinned host inputs -> device, GEMM, D -> pinned host
     e2e = None
@@ -411,11 +425,7 @@ def run_ours(args, rank: int, world: int) -> None:
                 e2e_step()
             s1.record(stream)
             torch.cuda.synchronize(dev)
-        e2e_ms = s0.elapsed_time(s1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, world, dev)
         e2e = {"value": world * acc["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": int(sum(v.nbytes for v in pin.values())),
                "d2h_bytes_per_step": int(d_host.nbytes), "steps": n_e2e,
@@ -448,7 +458,7 @@ def run_ours(args, rank: int, world: int) -> None:
     if kernels_per_call(variant) > 1:
         roof["launch_time_source"] += " (a call is the partial-sums kernel and its reduce kernel)"
 
-    value = world * acc["flops"] * args.steps / (ms_max * 1e-3) / 1e12
+    value = whole_job_tflops(world, acc["flops"], args.steps, ms_max)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
