@@ -11,7 +11,8 @@
 //
 //   warps 0, 3    TMA producers: for every (tile, K-block) one stage of a
 //                 shared-memory ring receives the 128-row "lane" operand
-//                 tile, the "column" operand tile and the tile's slice of sa.
+//                 tile, the "column" operand tile and (n-lanes only) the
+//                 tile's slice of sa.
 //                 Lanes 0..3 of both warps issue; stage s belongs to issuer
 //                 s % 8 for every round (one thread issues only about one
 //                 TMA operation per 150 ns, which would cap a CTA near
@@ -21,16 +22,19 @@
 //                 the K-block partial P_kb, FP32, into one of several
 //                 tensor-memory (TMEM) buffers; tcgen05.commit frees the
 //                 stage and signals the partial.  A single thread spends
-//                 about 650 cycles per K-block on waits, MMA issue and
-//                 commits, more than an N <= 128 MMA takes to execute; two
-//                 issuers overlap that work.
+//                 several hundred cycles per K-block on waits, MMA issue
+//                 and commits, more than an N <= 128 MMA takes to execute;
+//                 two issuers overlap that work.
 //   warps 4..11   two promotion warpgroups, each owning half the tile's
 //                 columns: tcgen05.ld the finished partial, acc += P * scale
 //                 in FP32 registers (CUDA cores), release the TMEM buffer so
 //                 the MMA of a later K-block overlaps; after the tile's last
-//                 K-block, round to bf16 and store D.  The sb values of the
-//                 tile are prefetched 32 K-blocks at a time into a register
-//                 per lane and broadcast with a shuffle.
+//                 K-block, round to bf16 and store D.  m-lanes: the thread's
+//                 scale sa[kb][m] * sb[g][nb][kb] is loaded from global
+//                 memory two K-blocks ahead; n-lanes: the per-column sa comes
+//                 with the stage and sb is prefetched 32 K-blocks at a time
+//                 into a register per lane and broadcast with a shuffle.
+//                 TMEM buffers are released with relaxed arrives.
 //
 // Orientation.  The MMA's M side (TMEM lanes) is always 128 rows.
 //   kSwap = true : lanes are 128 rows of B (n), columns are BNC rows of A
@@ -48,6 +52,11 @@
 // tile, each over K/SPLIT.  Each CTA stores its partial sums into the shared
 // memory of the CTA that owns those columns; after one cluster barrier every
 // CTA adds the SPLIT partials of its columns in rank order (deterministic).
+// SPLIT < 0 (global split-K): gsplit CTAs per tile store FP32 partials to a
+// workspace; either the CTAs of the tile reduce them after an arrival count
+// (kGlobalSplit) or splitk_reduce_kernel, launched next, does
+// (kGlobalSplitPartials).  HALF: see Layout.
+// The CTA-pair kernel (tcgen05 cta_group::2) is in kernel_pair.cuh.
 //
 // Programmatic dependent launch: the prologue (barrier init, TMEM
 // allocation, tensor-map prefetch) runs before griddepcontrol.wait, so it can
