@@ -113,3 +113,13 @@ def test_status_strings_and_variant_table(lib):
     assert lib.fp8g_set_variant_override(0) == 0
     assert lib.fp8g_set_variant_override(-1) == 0
     assert lib.fp8g_version() >= 100
+
+
+def test_every_variant_name_starts_with_its_kind(lib):
+    # the GPU parity tests run every variant whose name starts with the
+    # call's kind; a variant outside the three prefixes would go untested
+    names = [lib.fp8g_variant_name(i).decode() for i in range(lib.fp8g_num_variants())]
+    for n in names:
+        assert n.split("_", 1)[0] in ("dense", "contiguous", "masked"), n
+    for kind in ("dense", "contiguous", "masked"):
+        assert any(n.startswith(kind + "_") for n in names), kind
