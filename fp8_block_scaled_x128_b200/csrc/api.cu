@@ -321,7 +321,7 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
 
   const int KB = P.K / 128, NB = (P.N + 127) / 128;
   // output tile: n-lanes BNC rows of A x 128 rows of B; m-lanes 128 x BNC;
-  // pairs 256 x 256 (each CTA loads 128 rows of A and 128 rows of B)
+  // pairs 256 x BNC (each CTA loads 128 rows of A and BNC / 2 rows of B)
   const int m_ext = V.pair ? 256 : V.swap ? V.bnc : 128;
   const int n_ext = V.pair ? V.bnc : V.swap ? 128 : V.bnc;
   const int G_a = P.kind == kMasked ? P.G : 1;
@@ -460,8 +460,10 @@ int select_variant(const Problem& P, DeviceInfo* dev, cudaStream_t stream) {
     return wide(V_MASKED_M256, V_MASKED_M128, static_cast<long>(P.G) * m_blocks * ((P.N + 255) / 256));
   }
   if (P.M <= 64) {
-    // decode shapes: few 128-row tiles of B.  Split K over a cluster so that
-    // many SMs stream B; take the largest split whose clusters are all
+    // decode shapes: few 128-row tiles of B, so K is split for many SMs to
+    // stream B.  First choice: up to 16 CTAs per tile with partials in the
+    // workspace and a reduce kernel.  Without the workspace (a capture before
+    // the device's first call): a cluster split whose clusters are all
     // co-resident and that leaves each CTA at least 4 K-blocks.
     const int nt = (P.N + 127) / 128;
     const int kb = P.K / 128;
