@@ -6,8 +6,13 @@
 
 One step = one call of the GEMM over one batch of seeded synthetic input (all
 of the path: TMA tile loads, FP8 MMA per K-block, FP32 promotion, tile
-scheduling, bf16 epilogue).  The default workload is the dense decode shape
-M=64, N=2112, K=7168.
+scheduling, bf16 epilogue).  The default (headline) workload is the largest
+single-GPU configuration of the benchmark table: the contiguous M-grouped
+GEMM with 4 experts of 8192 rows, N=4096, K=7168.  The metric is per shape,
+so the same JSON line also carries a `per_shape` object with every workload
+of the table (dense 128x256x512, dense 64x2112x7168, dense 4096x7168x16384,
+contiguous, masked G=16), each timed in the same run with its own roofline,
+clock record and CPU-oracle baseline.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 device synchronise on both sides, timed with CUDA events on the launching
@@ -43,7 +48,7 @@ from fp8_block_scaled_x128_b200 import synth  # noqa: E402
 
 METRIC = "FP8 TFLOPS (bf16 out) and % of B200 FP8/HBM roofline per shape, 1 GPU"
 UNIT = "TFLOPS"
-DEFAULT_WORKLOAD = "dense_64x2112x7168"
+DEFAULT_WORKLOAD = "contiguous_g4_m8192_n4096_k7168"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 : BF16 tensor throughput (4.5 : 2.25 PFLOP/s)
@@ -261,7 +266,10 @@ def run_reference(args, rank: int, world: int) -> None:
     flop_per_row = acc["flops"] / max(1, acc["rows"])
     nthreads = oracle.default_threads()
     n1, dt1 = oracle_rows_per_second(d, nthreads, nthreads)  # one row per thread
-    per_step_rows = max(1, int(min(acc["rows"], n1 * 1.5 / max(dt1, 1e-6))))  # ~1.5 s per step
+    # each step a bounded sample: about 1.5 s, less when there are many steps,
+    # so that the whole run (warm-up included) takes about a minute at most
+    step_s = min(1.5, max(0.2, 60.0 / (args.steps + args.warmup)))
+    per_step_rows = max(1, int(min(acc["rows"], n1 * step_s / max(dt1, 1e-6))))
     for _ in range(args.warmup):
         oracle_rows_per_second(d, per_step_rows, nthreads)
     total_rows, total_t = 0, 0.0
@@ -284,53 +292,65 @@ def run_reference(args, rank: int, world: int) -> None:
 
 # --------------------------------------------------------------------------- GPU arm
 
-def run_ours(args, rank: int, world: int) -> None:
+# timed launches per shape in the per_shape block (at least --steps): enough
+# that each shape's timed region lasts ~10 ms or more
+PER_SHAPE_STEPS = {"dense_128x256x512": 400, "dense_64x2112x7168": 400, "dense_4096x7168x16384": 20,
+                   "contiguous_g4_m8192_n4096_k7168": 10, "masked_g16_m256_n4096_k7168": 60}
+
+
+class Shape:
+    """One workload on the device: inputs (rotated over enough copies that each
+    step reads HBM), output, and a step function calling the C ABI."""
+
+    def __init__(self, name: str, rank: int, dev):
+        import torch
+        from fp8_block_scaled_x128_b200 import gemm
+        self.gemm = gemm
+        self.name = name
+        self.dev = dev
+        d = workload_inputs(name, rank)
+        d["name"] = name
+        self.d = d
+        self.acc = accounting(d)
+        self.kind = d["kind"]
+        self.per_copy = input_bytes(d)
+        self.copies = 1 if self.per_copy >= 2 * L2_BYTES else int(math.ceil(2 * L2_BYTES / self.per_copy))
+        self.host = {k: torch.from_numpy(np.ascontiguousarray(d[k])) for k in ("A", "sa", "B", "sb")}
+        if self.kind == "contiguous":
+            self.host["idx"] = torch.from_numpy(d["m_indices"])
+        elif self.kind == "masked":
+            self.host["idx"] = torch.from_numpy(d["masked_m"])
+        self.sets = [{k: v.to(dev) for k, v in self.host.items()} for _ in range(self.copies)]
+        self.out_shape = (d["G"], d["Mmax"], d["N"]) if self.kind == "masked" else (d["M"], d["N"])
+        self.D = torch.empty(self.out_shape, dtype=torch.bfloat16, device=dev)
+
+    def step(self, i: int, stream):
+        g, t, d = self.gemm, self.sets[i % self.copies], self.d
+        if self.kind == "dense":
+            g.fp8_gemm_nt(t["A"], t["sa"], t["B"], t["sb"], D=self.D, stream=stream)
+        elif self.kind == "contiguous":
+            g.m_grouped_fp8_gemm_nt_contiguous(t["A"], t["sa"], t["B"], t["sb"], t["idx"], D=self.D, stream=stream)
+        else:
+            g.m_grouped_fp8_gemm_nt_masked(t["A"], t["sa"], t["B"], t["sb"], t["idx"], d["expected_m"], D=self.D,
+                                           stream=stream)
+
+    def l2_note(self) -> str:
+        if self.copies > 1:
+            return f"inputs rotate over {self.copies} device copies ({self.copies * self.per_copy / 2**20:.0f} MiB > 2x L2)"
+        return f"inputs {self.per_copy / 2**20:.0f} MiB >= 2x L2"
+
+
+def time_shape(S: Shape, steps: int, warmup: int, stream, sampler, world: int, per_launch_events: bool):
+    """Device time of `steps` back-to-back calls replayed from one CUDA graph,
+    bracketed by a barrier and a synchronise on both sides (max over ranks).
+    Returns (ms, per-launch ms list, clock summary, variant name)."""
     import torch
     import torch.distributed as dist
-
-    from fp8_block_scaled_x128_b200 import gemm
-
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-    torch.cuda.set_device(dev)
-    d = workload_inputs(args.workload, rank)
-    d["name"] = args.workload
-    acc = accounting(d)
-    kind = d["kind"]
-    if args.variant is not None:
-        gemm.set_variant_override(args.variant)
-
-    # device inputs, rotated through enough copies that each step reads HBM
-    per_copy = input_bytes(d)
-    copies = 1 if per_copy >= 2 * L2_BYTES else int(math.ceil(2 * L2_BYTES / per_copy))
-    host = {k: torch.from_numpy(np.ascontiguousarray(d[k])) for k in ("A", "sa", "B", "sb")}
-    if kind == "contiguous":
-        host["idx"] = torch.from_numpy(d["m_indices"])
-    elif kind == "masked":
-        host["idx"] = torch.from_numpy(d["masked_m"])
-    sets = [{k: v.to(dev) for k, v in host.items()} for _ in range(copies)]
-    if kind == "dense":
-        out_shape = (d["M"], d["N"])
-    elif kind == "contiguous":
-        out_shape = (d["M"], d["N"])
-    else:
-        out_shape = (d["G"], d["Mmax"], d["N"])
-    D = torch.empty(out_shape, dtype=torch.bfloat16, device=dev)
-
-    def step(i: int, s=None):
-        t = sets[i % copies]
-        if kind == "dense":
-            gemm.fp8_gemm_nt(t["A"], t["sa"], t["B"], t["sb"], D=D, stream=s)
-        elif kind == "contiguous":
-            gemm.m_grouped_fp8_gemm_nt_contiguous(t["A"], t["sa"], t["B"], t["sb"], t["idx"], D=D, stream=s)
-        else:
-            gemm.m_grouped_fp8_gemm_nt_masked(t["A"], t["sa"], t["B"], t["sb"], t["idx"], d["expected_m"], D=D,
-                                              stream=s)
-
-    stream = torch.cuda.Stream(device=dev)
+    dev = S.dev
     with torch.cuda.stream(stream):
-        step(0, stream)  # per-device set-up outside capture
+        S.step(0, stream)  # per-device set-up outside capture
     torch.cuda.synchronize(dev)
-    variant = gemm.variant_names()[gemm.last_variant()]
+    variant = S.gemm.variant_names()[S.gemm.last_variant()]
 
     def capture(nsteps: int, first: int, events: bool):
         g = torch.cuda.CUDAGraph()
@@ -339,21 +359,18 @@ def run_ours(args, rank: int, world: int) -> None:
             for i in range(nsteps):
                 if events:
                     evs[i].record(stream)
-                step(first + i, stream)
+                S.step(first + i, stream)
             if events:
                 evs[nsteps].record(stream)
         return g, evs
 
-    warm_graph, _ = capture(max(1, args.warmup), 0, False)
+    warm_graph, _ = capture(max(1, warmup), 0, False)
     # no event nodes between the timed launches: they would stop a launch
     # from overlapping its prologue with the previous one (programmatic
     # dependent launch); the average launch time is the region time / K
-    timed_graph, evs = capture(args.steps, args.warmup, args.per_launch_events)
+    timed_graph, evs = capture(steps, warmup, per_launch_events)
 
-    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    sampler = ClockSampler(gpu_id) if not args.no_clocks else ClockSampler.disabled()
-
-    def timed_region():
+    def region():
         # graph.replay() launches on torch's current stream: make it `stream`,
         # the stream the timing events are recorded on
         with torch.cuda.stream(stream):
@@ -380,64 +397,26 @@ def run_ours(args, rank: int, world: int) -> None:
             dist.barrier()
         t_end = time.time()
         ms = start.elapsed_time(end)
-        if args.per_launch_events:
-            per_launch = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
-        else:
-            per_launch = [ms / args.steps] * args.steps
+        per_launch = ([evs[i].elapsed_time(evs[i + 1]) for i in range(steps)] if per_launch_events
+                      else [ms / steps] * steps)
         return ms, per_launch, sampler.summary(soak_t0, t_end)
 
-    time.sleep(0.5)
-    ms, per_launch, clocks = timed_region()
-    remeasured = False
+    ms, per_launch, clocks = region()
     if clocks_rejected(clocks):
-        ms, per_launch, clocks = timed_region()
-        remeasured = True
-    sampler.stop()
-    err = gemm.device_error(clear=True)
+        ms, per_launch, clocks = region()
+        if clocks is not None:
+            clocks["remeasured"] = True
+    err = S.gemm.device_error(clear=True)
     if err:
-        raise RuntimeError(f"device error word {err:#x} after the timed region")
+        raise RuntimeError(f"device error word {err:#x} after the timed region of {S.name}")
+    del warm_graph, timed_graph
+    return ms, per_launch, clocks, variant
 
-    ms_max = max_over_ranks(ms, world, dev)
 
-    # end to end through the public API: pinned host inputs -> device, GEMM, D -> pinned host
-    e2e = None
-    if not args.no_e2e:
-        pin = {k: v.pin_memory() for k, v in host.items()}
-        dev_in = sets[0]
-        d_host = torch.empty(out_shape, dtype=torch.bfloat16).pin_memory()
-        n_e2e = max(3, min(args.steps, 50))
-
-        def e2e_step():
-            for k in pin:
-                dev_in[k].copy_(pin[k], non_blocking=True)
-            step(0, stream)
-            d_host.copy_(D, non_blocking=True)
-
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                e2e_step()
-            torch.cuda.synchronize(dev)
-            if world > 1:
-                dist.barrier()
-            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s0.record(stream)
-            for _ in range(n_e2e):
-                e2e_step()
-            s1.record(stream)
-            torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, world, dev)
-        e2e = {"value": world * acc["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": int(sum(v.nbytes for v in pin.values())),
-               "d2h_bytes_per_step": int(d_host.nbytes), "steps": n_e2e,
-               "note": "pinned host inputs copied to the device, GEMM through the C ABI, D copied back, every step"}
-
-    if rank != 0:
-        return
-
+def roofline(acc, avg_launch_s: float, workload: str, variant: str, per_launch_events: bool) -> dict:
     pk = peaks()
     ridge = pk["bf16"] * FP8_OVER_BF16 * 1e12 / (pk["hbm"] * 1e9)
     intensity = acc["flops"] / acc["bytes"]
-    avg_launch_s = statistics.mean(per_launch) * 1e-3
     if intensity < ridge:
         achieved = acc["bytes"] / avg_launch_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
@@ -448,35 +427,132 @@ def run_ours(args, rank: int, world: int) -> None:
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak,
                 "peak_source": f"bf16_tflops (burst) of {pk['source']} x {FP8_OVER_BF16} (FP8:BF16 nominal)"}
-    roof["traffic"] = ncu_traffic(args.workload, variant)
+    roof["traffic"] = ncu_traffic(workload, variant)
     roof["kernel"] = variant
     roof["algorithmic_bytes_per_launch"] = acc["bytes"]
     roof["algorithmic_flops_per_launch"] = acc["flops"]
     roof["avg_launch_us"] = avg_launch_s * 1e6
-    roof["launch_time_source"] = ("CUDA events around every launch" if args.per_launch_events else
+    roof["launch_time_source"] = ("CUDA events around every launch" if per_launch_events else
                                   "CUDA events around the K back-to-back launches of the timed region, / K")
     if kernels_per_call(variant) > 1:
         roof["launch_time_source"] += " (a call is the partial-sums kernel and its reduce kernel)"
+    return roof
 
-    value = whole_job_tflops(world, acc["flops"], args.steps, ms_max)
+
+def e2e_measure(S: Shape, steps: int, stream, world: int) -> dict:
+    """The same metric end to end through the public API: pinned host inputs
+    copied to the device, the C-ABI call, D copied back to pinned host memory,
+    every step."""
+    import torch
+    import torch.distributed as dist
+    dev = S.dev
+    pin = {k: v.pin_memory() for k, v in S.host.items()}
+    dev_in = S.sets[0]
+    d_host = torch.empty(S.out_shape, dtype=torch.bfloat16).pin_memory()
+    n_e2e = max(3, min(steps, 50))
+
+    def e2e_step():
+        for k in pin:
+            dev_in[k].copy_(pin[k], non_blocking=True)
+        S.step(0, stream)
+        d_host.copy_(S.D, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, world, dev)
+    return {"value": world * S.acc["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+            "h2d_bytes_per_step": int(sum(v.nbytes for v in pin.values())),
+            "d2h_bytes_per_step": int(d_host.nbytes), "steps": n_e2e,
+            "note": "pinned host inputs copied to the device, GEMM through the C ABI, D copied back, every step"}
+
+
+def run_ours(args, rank: int, world: int) -> None:
+    import torch
+
+    from fp8_block_scaled_x128_b200 import gemm
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    if args.variant is not None:
+        gemm.set_variant_override(args.variant)
+    stream = torch.cuda.Stream(device=dev)
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_id) if not args.no_clocks else ClockSampler.disabled()
+    time.sleep(0.5)
+    with_cpu = world == 1 and rank == 0 and not args.no_cpu_baseline
+    try:
+        # the headline workload: exactly --steps timed steps, e2e, oracle baseline
+        S = Shape(args.workload, rank, dev)
+        ms, per_launch, clocks, variant = time_shape(S, args.steps, args.warmup, stream, sampler, world,
+                                                     args.per_launch_events)
+        ms_max = max_over_ranks(ms, world, dev)
+        e2e = None if args.no_e2e else e2e_measure(S, args.steps, stream, world)
+        head = dict(S=S, ms=ms_max, per_launch=per_launch, clocks=clocks, variant=variant)
+        headline_cpu = cpu_baseline(S.d) if with_cpu else None
+        head_acc, head_d, head_l2 = S.acc, S.d, S.l2_note()
+        del S
+        torch.cuda.empty_cache()
+
+        # every workload of the benchmark table, measured in the same run
+        per_shape = {}
+        if not args.no_per_shape:
+            for name in synth.CONFIGS:
+                if name == args.workload:
+                    ps_ms, ps_launch, ps_clocks, ps_variant, ps_steps, acc = (
+                        ms_max, per_launch, clocks, variant, args.steps, head_acc)
+                    ps_cpu = headline_cpu
+                else:
+                    S = Shape(name, rank, dev)
+                    ps_steps = max(args.steps, PER_SHAPE_STEPS.get(name, args.steps))
+                    ps_ms, ps_launch, ps_clocks, ps_variant = time_shape(S, ps_steps, args.warmup, stream, sampler,
+                                                                         world, args.per_launch_events)
+                    ps_ms = max_over_ranks(ps_ms, world, dev)
+                    acc = S.acc
+                    ps_cpu = cpu_baseline(S.d, target_s=4.0) if with_cpu else None
+                    del S
+                    torch.cuda.empty_cache()
+                avg_s = ps_ms / ps_steps * 1e-3
+                per_shape[name] = {
+                    "value": whole_job_tflops(world, acc["flops"], ps_steps, ps_ms), "unit": UNIT,
+                    "us_per_launch": avg_s * 1e6, "steps": ps_steps, "variant": ps_variant,
+                    "roofline": roofline(acc, avg_s, name, ps_variant, args.per_launch_events),
+                    "gpu_launches": world * ps_steps * kernels_per_call(ps_variant),
+                    "clocks": ps_clocks, "cpu_baseline": ps_cpu,
+                }
+    finally:
+        sampler.stop()
+
+    if rank != 0:
+        return
+    avg_launch_s = statistics.mean(head["per_launch"]) * 1e-3
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "metric": METRIC, "value": whole_job_tflops(world, head_acc["flops"], args.steps, head["ms"]), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms"] / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
         "data": "synthetic (seeded generator: bf16 N(0,1) draws quantised to e4m3 with 1x128 / 128x128 FP32 scales)",
-        "config": {"workload": args.workload, "shape": {k: d[k] for k in ("M", "N", "K", "G", "Mmax") if k in d},
-                   "accumulate": "fp32 (per-128-K-block promotion)", "out": "bf16",
-                   "l2": (f"inputs rotate over {copies} device copies ({copies * per_copy / 2**20:.0f} MiB > 2x L2)"
-                          if copies > 1 else f"inputs {per_copy / 2**20:.0f} MiB >= 2x L2"),
+        "config": {"workload": args.workload,
+                   "shape": {k: head_d[k] for k in ("M", "N", "K", "G", "Mmax") if k in head_d},
+                   "accumulate": "fp32 (per-128-K-block promotion)", "out": "bf16", "l2": head_l2,
                    "launch": "CUDA graph of the K steps, one C-ABI call each",
-                   "variant": variant, "parallelism": "replicas" if world > 1 else "single GPU"},
-        "roofline": roof, "gpu_launches": world * args.steps * kernels_per_call(variant), "clocks": clocks,
+                   "variant": head["variant"], "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": roofline(head_acc, avg_launch_s, args.workload, head["variant"], args.per_launch_events),
+        "gpu_launches": world * args.steps * kernels_per_call(head["variant"]), "clocks": head["clocks"],
         "e2e": e2e,
     }
-    if remeasured:
-        line["clocks_remeasured"] = True
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(d)
+    if headline_cpu is not None:
+        line["cpu_baseline"] = headline_cpu
+    if per_shape:
+        line["per_shape"] = per_shape
     print(json.dumps(line), flush=True)
 
 
@@ -490,6 +566,7 @@ def main() -> int:
     ap.add_argument("--variant", type=int, default=None, help="force a kernel variant (tuning)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-shape", action="store_true", help="measure the headline workload only")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi clocks (diagnostic)")
     ap.add_argument("--per-launch-events", action="store_true",
                     help="record an event between launches (diagnostic; prevents launch overlap)")

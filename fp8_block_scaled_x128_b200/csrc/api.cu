@@ -35,11 +35,11 @@ struct Variant {
   int launch_regs;  // register-split variants: registers per thread at launch
 };
 
-template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int MINB = 1, bool HALF = false>
+template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT>
 Variant make_variant(const char* name) {
-  using L = Layout<kSwap, BNC, STAGES, SPLIT, MINB, HALF>;
+  using L = Layout<kSwap, BNC, STAGES, SPLIT>;
   return Variant{name, KIND, kSwap, BNC, STAGES, SPLIT, L::kRegSplit,
-                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT, MINB, HALF>, L::kSmemAlloc, false,
+                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT>, L::kSmemAlloc, false,
                  kThreads, kLaunchRegs};
 }
 
@@ -50,71 +50,44 @@ Variant make_pair_variant(const char* name) {
 }
 
 // "nlanes": TMEM lanes are rows of B (small M); "mlanes": lanes are rows of A.
+// Every entry is reachable: select_variant picks it for some call, or it is
+// the fallback of one (cluster split-K without a workspace, single-CTA tiles
+// when too few pair tiles fill the GPU), or fp8_gemm_nt_no_alloc runs it.
 const Variant kVariants[] = {
     make_variant<true, 64, 6, kDense, 8>("dense_nlanes_bn64_st6_splitk8"),
-    make_variant<true, 64, 8, kDense, 1>("dense_nlanes_bn64_st8"),
-    make_variant<true, 128, 6, kDense, 1>("dense_nlanes_bn128_st6"),
-    make_variant<false, 128, 6, kDense, 1>("dense_mlanes_bn128_st6"),
-    make_variant<true, 128, 6, kContiguous, 1>("contiguous_nlanes_bn128_st6"),
-    make_variant<false, 128, 6, kContiguous, 1>("contiguous_mlanes_bn128_st6"),
-    make_variant<true, 64, 8, kMasked, 1>("masked_nlanes_bn64_st8"),
-    make_variant<true, 128, 6, kMasked, 1>("masked_nlanes_bn128_st6"),
-    make_variant<false, 128, 6, kMasked, 1>("masked_mlanes_bn128_st6"),
     make_variant<true, 64, 6, kDense, 4>("dense_nlanes_bn64_st6_splitk4"),
     make_variant<true, 64, 6, kDense, 2>("dense_nlanes_bn64_st6_splitk2"),
-    make_variant<false, 256, 4, kDense, 1>("dense_mlanes_bn256_st4"),
-    make_variant<false, 256, 4, kContiguous, 1>("contiguous_mlanes_bn256_st4"),
-    make_variant<false, 256, 4, kMasked, 1>("masked_mlanes_bn256_st4"),
+    make_variant<true, 64, 8, kDense, 1>("dense_nlanes_bn64_st8"),
     make_variant<true, 64, 8, kDense, kGlobalSplit>("dense_nlanes_bn64_st8_gsplit"),
     make_variant<true, 64, 8, kDense, kGlobalSplitPartials>("dense_nlanes_bn64_st8_gsplit_2k"),
-    make_variant<true, 64, 4, kDense, kGlobalSplitPartials, 2>("dense_nlanes_bn64_st4_gsplit_2k_x2"),
-    make_pair_variant<kDense, 6, 256>("dense_mlanes_pair_bn256_st6"),
-    make_pair_variant<kMasked, 6, 256>("masked_mlanes_pair_bn256_st6"),
-    make_variant<false, 256, 4, kDense, 1, 1, true>("dense_mlanes_bn256h_st4"),
-    make_variant<false, 256, 4, kContiguous, 1, 1, true>("contiguous_mlanes_bn256h_st4"),
-    make_variant<false, 256, 4, kMasked, 1, 1, true>("masked_mlanes_bn256h_st4"),
-    make_pair_variant<kDense, 6, 192>("dense_mlanes_pair_bn192_st6"),
-    make_pair_variant<kMasked, 6, 192>("masked_mlanes_pair_bn192_st6"),
-    make_pair_variant<kContiguous, 6, 192>("contiguous_mlanes_pair_bn192_st6"),
-    make_pair_variant<kDense, 8, 128>("dense_mlanes_pair_bn128_st8"),
-    make_pair_variant<kContiguous, 8, 128>("contiguous_mlanes_pair_bn128_st8"),
-    make_pair_variant<kMasked, 8, 128>("masked_mlanes_pair_bn128_st8"),
+    make_variant<false, 128, 6, kDense, 1>("dense_mlanes_bn128_st6"),
+    make_variant<false, 256, 4, kDense, 1>("dense_mlanes_bn256_st4"),
     make_pair_variant<kDense, 8, 192>("dense_mlanes_pair_bn192_st8"),
-    make_pair_variant<kMasked, 8, 192>("masked_mlanes_pair_bn192_st8"),
+    make_variant<false, 128, 6, kContiguous, 1>("contiguous_mlanes_bn128_st6"),
+    make_variant<false, 256, 4, kContiguous, 1>("contiguous_mlanes_bn256_st4"),
+    make_variant<false, 128, 6, kMasked, 1>("masked_mlanes_bn128_st6"),
+    make_variant<false, 256, 4, kMasked, 1>("masked_mlanes_bn256_st4"),
+    make_pair_variant<kMasked, 6, 192>("masked_mlanes_pair_bn192_st6"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
   V_DENSE_SPLIT = 0,
-  V_DENSE_N64 = 1,
-  V_DENSE_N128 = 2,
-  V_DENSE_M128 = 3,
-  V_CONTIG_N128 = 4,
-  V_CONTIG_M128 = 5,
-  V_MASKED_N64 = 6,
-  V_MASKED_N128 = 7,
-  V_MASKED_M128 = 8,
-  V_DENSE_SPLIT4 = 9,
-  V_DENSE_SPLIT2 = 10,
-  V_DENSE_M256 = 11,
-  V_CONTIG_M256 = 12,
-  V_MASKED_M256 = 13,
-  V_DENSE_GSPLIT = 14,
-  V_DENSE_GSPLIT2K = 15,
-  V_DENSE_GSPLIT2K_X2 = 16,
-  V_DENSE_PAIR = 17,
-  V_MASKED_PAIR = 18,
-  V_DENSE_M256H = 19,
-  V_CONTIG_M256H = 20,
-  V_MASKED_M256H = 21,
-  V_DENSE_PAIR192 = 22,
-  V_MASKED_PAIR192 = 23,
-  V_CONTIG_PAIR192 = 24,
-  V_DENSE_PAIR128 = 25,
-  V_CONTIG_PAIR128 = 26,
-  V_MASKED_PAIR128 = 27,
-  V_DENSE_PAIR192_S8 = 28,
-  V_MASKED_PAIR192_S8 = 29,
+  V_DENSE_SPLIT4,
+  V_DENSE_SPLIT2,
+  V_DENSE_N64,
+  V_DENSE_GSPLIT,
+  V_DENSE_GSPLIT2K,
+  V_DENSE_M128,
+  V_DENSE_M256,
+  V_DENSE_PAIR192_S8,
+  V_CONTIG_M128,
+  V_CONTIG_M256,
+  V_MASKED_M128,
+  V_MASKED_M256,
+  V_MASKED_PAIR192,
+  V_COUNT
 };
+static_assert(V_COUNT == kNumVariants, "variant table and names");
 
 std::atomic<int> g_override{-1};
 
@@ -530,6 +503,21 @@ int m_grouped_fp8_gemm_nt_masked(const uint8_t* A, const float* sa, int ld_sa, c
   return run(Problem{kMasked, A, sa, ld_sa, B, sb, D, masked_m, Mmax, N, K, G, expected_m}, stream);
 }
 
+int fp8g_sa_to_mn_major(const float* src, float* dst, int G, int rows, int KB, int ld_sa) {
+  if (!src || !dst || G < 1 || rows < 0 || KB < 1 || ld_sa < rows || ld_sa < 1) return FP8G_ERR_INVALID_ARG;
+  if (ld_sa % 4 != 0) return FP8G_ERR_MISALIGNED;
+  for (long g = 0; g < G; ++g) {
+    const float* s = src + g * rows * static_cast<long>(KB);
+    float* d = dst + g * KB * static_cast<long>(ld_sa);
+    for (long kb = 0; kb < KB; ++kb) {
+      float* drow = d + kb * ld_sa;
+      for (long m = 0; m < rows; ++m) drow[m] = s[m * KB + kb];
+      for (long m = rows; m < ld_sa; ++m) drow[m] = 0.f;
+    }
+  }
+  return FP8G_OK;
+}
+
 const char* fp8g_status_string(int status) {
   switch (status) {
     case FP8G_OK: return "ok";
@@ -591,10 +579,9 @@ int fp8g_version(void) { return 100; }
 // device memory.
 //
 // Some callers cannot call cudaMalloc at the point where they run a GEMM: an
-// engine that hands out all device memory from its own fixed pool, code that
-// runs while another component is capturing a CUDA graph (an allocation
-// there would break the capture), or a runtime that forbids allocations
-// after start-up so that its memory footprint is known in advance.  The
+// engine that hands out all device memory from its own fixed pool, or a
+// runtime that forbids allocations after start-up so that its memory
+// footprint is known in advance.  The
 // regular fp8_gemm_nt allocates its split-K workspace (about 4.7 MB) on the
 // first decode-shaped call of a device.  This entry point runs the same
 // split-K kernel with its scratch in a statically sized array that the

@@ -55,7 +55,7 @@
 // SPLIT < 0 (global split-K): gsplit CTAs per tile store FP32 partials to a
 // workspace; either the CTAs of the tile reduce them after an arrival count
 // (kGlobalSplit) or splitk_reduce_kernel, launched next, does
-// (kGlobalSplitPartials).  HALF: see Layout.
+// (kGlobalSplitPartials).
 // The CTA-pair kernel (tcgen05 cta_group::2) is in kernel_pair.cuh.
 //
 // Programmatic dependent launch: the prologue (barrier init, TMEM
@@ -128,20 +128,12 @@ constexpr int pow2_at_least(int x, int lo) {
   return p;
 }
 
-// MINB: CTAs that must fit on one SM together (2 lets the next launch's
-// CTAs start their prologue beside a running CTA: half the TMEM and shared
-// memory, and at most 85 registers per thread).
-// HALF (m-lanes, BNC = 256): each K-block's MMA is issued as two N = 128
-// halves into separate 128-column TMEM slots with their own commits, so each
-// promotion warpgroup waits only for its own half and the MMA may refill a
-// slot while the other half of the same buffer is still being read.
-template <bool kSwap, int BNC, int STAGES, int SPLIT, int MINB = 1, bool HALF = false>
+template <bool kSwap, int BNC, int STAGES, int SPLIT>
 struct Layout {
   static constexpr int kLaneBytes = 128 * 128;   // 128 rows x 128 e4m3 (one K-block)
   static constexpr int kColBytes = BNC * 128;
   static constexpr int kSaFloats = kSwap ? BNC : 0;  // sa slice (n-lanes only): the tile's m-extent
-  static constexpr int kTmemBudget = 512 / MINB;
-  static constexpr int kNBuf = kTmemBudget / BNC < 8 ? kTmemBudget / BNC : 8;  // TMEM partial buffers
+  static constexpr int kNBuf = 512 / BNC < 8 ? 512 / BNC : 8;  // TMEM partial buffers
   static constexpr int kTmemCols = pow2_at_least(kNBuf * BNC, 32);
   static constexpr int kCW = BNC / 2;                  // columns per promotion warpgroup
   static constexpr bool kRegSplit = kCW > 64;          // 128 accumulators per thread
@@ -152,10 +144,7 @@ struct Layout {
   static constexpr int kOffRecv = kOffSa + STAGES * kSaFloats * 4;
   static constexpr int kRecvBytes = SPLIT > 1 ? SPLIT * 128 * kCPD * 4 : 0;
   static constexpr int kOffBar = kOffRecv + kRecvBytes;
-  static constexpr bool kHalf = HALF;
-  static constexpr int kSlots = HALF ? 2 * kNBuf : kNBuf;  // TMEM slots with their own full/empty barriers
-  static constexpr int kSlotCols = HALF ? BNC / 2 : BNC;
-  static constexpr int kNumBars = 2 * STAGES + 2 * kSlots + 2;
+  static constexpr int kNumBars = 2 * STAGES + 2 * kNBuf + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;  // + slack to align the base to 1024
@@ -170,9 +159,8 @@ struct Layout {
                 "cluster split-K layout");
   static_assert(SPLIT >= 1 || kSwap, "global split-K is for the n-lanes orientation");
   static_assert(!kRegSplit || !kSwap, "the register split is for the m-lanes orientation");
-  static_assert(kSmemAlloc <= 232448 && kSmemAlloc * MINB <= 231424, "shared memory");
+  static_assert(kSmemAlloc <= 232448, "shared memory");
   static_assert(kNBuf >= 2, "TMEM buffers");
-  static_assert(!HALF || (!kSwap && BNC == 256 && SPLIT == 1), "half-split MMA: m-lanes, 256 columns");
 };
 
 // Register budget of the BNC = 256 variants: 384 threads launch with 168
@@ -335,11 +323,11 @@ __device__ __forceinline__ void global_split_reduce(const Params& p, int tile, u
   }
 }
 
-template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int MINB = 1, bool HALF = false>
-__global__ void __launch_bounds__(kThreads, MINB)
+template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT>
+__global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSA, const Params p) {
-  using L = Layout<kSwap, BNC, STAGES, SPLIT, MINB, HALF>;
+  using L = Layout<kSwap, BNC, STAGES, SPLIT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -352,8 +340,8 @@ __global__ void __launch_bounds__(kThreads, MINB)
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + L::kSlots + b); };
-  auto drain_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + 2 * L::kSlots + i); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + L::kNBuf + b); };
+  auto drain_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + 2 * L::kNBuf + i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -370,10 +358,9 @@ __global__ void __launch_bounds__(kThreads, MINB)
       // MMA commit, plus the promotion warps where they read the stage's sa slice
       mbar_init(empty_bar(s), kSwap ? 1 + kPromoWarps : 1);
     }
-    for (int b = 0; b < L::kSlots; ++b) {
+    for (int b = 0; b < L::kNBuf; ++b) {
       mbar_init(tfull_bar(b), 1);
-      // a half slot is read by the four warps of one promotion warpgroup
-      mbar_init(tempty_bar(b), L::kHalf ? kPromoWarps / 2 : kPromoWarps);
+      mbar_init(tempty_bar(b), kPromoWarps);
     }
     mbar_init(drain_bar(0), 1);
     mbar_init(drain_bar(1), 1);
@@ -468,34 +455,6 @@ __global__ void __launch_bounds__(kThreads, MINB)
           const uint32_t ph = (it / STAGES) & 1u;
           const int b = it % L::kNBuf;
           const uint32_t tph = (it / L::kNBuf) & 1u;
-          if constexpr (L::kHalf) {
-            // two N = 128 halves: rows 0..127 and 128..255 of the column tile
-            // into slots 2b and 2b + 1, each committed on its own
-            if (!wait_phase(full_bar(s), ph, abort_flag)) {
-              ok = false;
-              break;
-            }
-            const uint64_t adesc = sdesc_k128_sw128(lane_tile(s));
-            constexpr uint32_t kIdescHalf = idesc_e4m3_f32(128, BNC / 2);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (!wait_phase(tempty_bar(2 * b + h), tph ^ 1u, abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BNC + h * (BNC / 2));
-              const uint64_t bdesc = sdesc_k128_sw128(col_tile(s) + static_cast<uint32_t>(h * (BNC / 2) * 128));
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_f8f6f4(d_tmem, adesc + static_cast<uint64_t>(2 * k), bdesc + static_cast<uint64_t>(2 * k),
-                           kIdescHalf, k > 0 ? 1u : 0u);
-              mma_commit(tfull_bar(2 * b + h));
-            }
-            if (!ok) break;
-            mma_commit(empty_bar(s));
-            continue;
-          }
           if (!wait_phase(full_bar(s), ph, abort_flag) ||
               !wait_phase(tempty_bar(b), tph ^ 1u, abort_flag)) {
             ok = false;
@@ -566,8 +525,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
             if (kb + u >= T.kb1) break;
             const int b = it % L::kNBuf;
             const uint32_t tph = (it / L::kNBuf) & 1u;
-            const int slot = L::kHalf ? 2 * b + wg : b;  // this warpgroup's barrier pair
-            if (!__all_sync(0xffffffffu, wait_phase(tfull_bar(slot), tph, abort_flag))) {
+            if (!__all_sync(0xffffffffu, wait_phase(tfull_bar(b), tph, abort_flag))) {
               ok = false;
               break;
             }
@@ -591,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_relaxed(tempty_bar(slot));
+            if (lane == 0) mbar_arrive_relaxed(tempty_bar(b));
             ++it;
           }
         }

@@ -30,6 +30,8 @@ lib.m_grouped_fp8_gemm_nt_masked.restype = _I
 lib.m_grouped_fp8_gemm_nt_masked.argtypes = [_P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 lib.fp8_gemm_nt_no_alloc.restype = _I
 lib.fp8_gemm_nt_no_alloc.argtypes = [_P, _P, _I, _P, _P, _P, _I, _I, _I, _P]
+lib.fp8g_sa_to_mn_major.restype = _I
+lib.fp8g_sa_to_mn_major.argtypes = [_P, _P, _I, _I, _I, _I]
 lib.fp8g_status_string.restype = C.c_char_p
 lib.fp8g_status_string.argtypes = [_I]
 lib.fp8g_get_device_error.restype = _I
@@ -63,8 +65,10 @@ def _ptr(t):
     return None if t is None else C.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
+def _stream(stream, device):
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    if s.device != device:
+        raise ValueError(f"stream is on {s.device}, the operands on {device}")
     return C.c_void_p(s.cuda_stream)
 
 
@@ -72,6 +76,19 @@ def _dev(t, dt, name):
     if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
         raise TypeError(f"{name}: expected a contiguous CUDA tensor of {dt}, got {t.dtype} on {t.device}")
     return t
+
+
+def _one_device(**tensors):
+    """The device every operand lives on.  The library encodes its tensor maps
+    and launches on the current device, so the call runs under this device and
+    operands on different devices are refused before anything is launched."""
+    devs = {name: t.device for name, t in tensors.items()}
+    first = next(iter(devs.values()))
+    for name, d in devs.items():
+        if d != first:
+            raise ValueError(f"all operands must be on one device: {name} is on {d}, "
+                             f"{next(iter(devs))} on {first}")
+    return first
 
 
 def variant_names():
@@ -106,8 +123,10 @@ def fp8_gemm_nt(A, sa, B, sb, D=None, stream=None):
     if D is None:
         D = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     _dev(D, torch.bfloat16, "D")
-    _check(lib.fp8_gemm_nt(_ptr(A), _ptr(sa), sa.shape[1], _ptr(B), _ptr(sb), _ptr(D), M, N, K,
-                           _stream(stream)), "fp8_gemm_nt")
+    dev = _one_device(A=A, sa=sa, B=B, sb=sb, D=D)
+    with torch.cuda.device(dev):
+        _check(lib.fp8_gemm_nt(_ptr(A), _ptr(sa), sa.shape[1], _ptr(B), _ptr(sb), _ptr(D), M, N, K,
+                               _stream(stream, dev)), "fp8_gemm_nt")
     return D
 
 
@@ -121,9 +140,11 @@ def m_grouped_fp8_gemm_nt_contiguous(A, sa, B, sb, m_indices, D=None, stream=Non
     if D is None:
         D = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     _dev(D, torch.bfloat16, "D")
-    _check(lib.m_grouped_fp8_gemm_nt_contiguous(_ptr(A), _ptr(sa), sa.shape[1], _ptr(B), _ptr(sb), _ptr(D),
-                                                _ptr(m_indices), M, N, K, G, _stream(stream)),
-           "m_grouped_fp8_gemm_nt_contiguous")
+    dev = _one_device(A=A, sa=sa, B=B, sb=sb, D=D, m_indices=m_indices)
+    with torch.cuda.device(dev):
+        _check(lib.m_grouped_fp8_gemm_nt_contiguous(_ptr(A), _ptr(sa), sa.shape[1], _ptr(B), _ptr(sb), _ptr(D),
+                                                    _ptr(m_indices), M, N, K, G, _stream(stream, dev)),
+               "m_grouped_fp8_gemm_nt_contiguous")
     return D
 
 
@@ -137,9 +158,11 @@ def m_grouped_fp8_gemm_nt_masked(A, sa, B, sb, masked_m, expected_m, D=None, str
     if D is None:
         D = torch.empty((G, Mmax, N), dtype=torch.bfloat16, device=A.device)
     _dev(D, torch.bfloat16, "D")
-    _check(lib.m_grouped_fp8_gemm_nt_masked(_ptr(A), _ptr(sa), sa.shape[2], _ptr(B), _ptr(sb), _ptr(D),
-                                            _ptr(masked_m), G, Mmax, N, K, int(expected_m),
-                                            _stream(stream)), "m_grouped_fp8_gemm_nt_masked")
+    dev = _one_device(A=A, sa=sa, B=B, sb=sb, D=D, masked_m=masked_m)
+    with torch.cuda.device(dev):
+        _check(lib.m_grouped_fp8_gemm_nt_masked(_ptr(A), _ptr(sa), sa.shape[2], _ptr(B), _ptr(sb), _ptr(D),
+                                                _ptr(masked_m), G, Mmax, N, K, int(expected_m),
+                                                _stream(stream, dev)), "m_grouped_fp8_gemm_nt_masked")
     return D
 
 
@@ -156,6 +179,25 @@ def fp8_gemm_nt_no_alloc(A, sa, B, sb, D=None, stream=None):
     if D is None:
         D = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     _dev(D, torch.bfloat16, "D")
-    _check(lib.fp8_gemm_nt_no_alloc(_ptr(A), _ptr(sa), sa.shape[1], _ptr(B), _ptr(sb), _ptr(D), M, N, K,
-                                    _stream(stream)), "fp8_gemm_nt_no_alloc")
+    dev = _one_device(A=A, sa=sa, B=B, sb=sb, D=D)
+    with torch.cuda.device(dev):
+        _check(lib.fp8_gemm_nt_no_alloc(_ptr(A), _ptr(sa), sa.shape[1], _ptr(B), _ptr(sb), _ptr(D), M, N, K,
+                                        _stream(stream, dev)), "fp8_gemm_nt_no_alloc")
     return D
+
+
+def sa_to_mn_major(sa_rows, ld_sa=None):
+    """Host helper: A's scales from [rows, KB] (or [G, rows, KB]) float32 to the
+    library's MN-major [KB, ld_sa] (or [G, KB, ld_sa]) layout, as a numpy array.
+    ld_sa defaults to rows rounded up to a multiple of 4."""
+    import numpy as np
+    src = np.ascontiguousarray(sa_rows, dtype=np.float32)
+    grouped = src.ndim == 3
+    if not grouped:
+        src = src[None]
+    G, rows, KB = src.shape
+    ld = max(4, (rows + 3) // 4 * 4) if ld_sa is None else int(ld_sa)
+    dst = np.empty((G, KB, ld), np.float32)
+    _check(lib.fp8g_sa_to_mn_major(src.ctypes.data_as(_P), dst.ctypes.data_as(_P), G, rows, KB, ld),
+           "fp8g_sa_to_mn_major")
+    return dst if grouped else dst[0]

@@ -35,14 +35,17 @@
  *      ld_sa >= M (Mmax for the masked call) and ld_sa % 4 == 0;
  *      A, B, sa, D 16-byte aligned; sb, m_indices, masked_m 4-byte aligned.
  *    M == 0 or N == 0 (or G == 0) is a no-op that returns FP8G_OK.
- *  - The call enqueues kernels on `stream` and returns without waiting.  It
- *    never reads device memory on the host, so it can be captured in a CUDA
- *    graph.  D is complete when the stream reaches that point.  The one
- *    exception to "never waits": see fp8_gemm_nt's workspace below.
+ *  - The call enqueues kernels on `stream` and returns without waiting; D is
+ *    complete when the stream reaches that point.  fp8_gemm_nt and the two
+ *    grouped calls never read device memory on the host, so they can be
+ *    captured in a CUDA graph.  The one exception to "never waits": see
+ *    fp8_gemm_nt's workspace below.
  *  - Errors found on the host come back as the return value; nothing is
  *    launched then.  Errors found by the kernel (a bad m_indices entry, a
  *    masked_m above Mmax, a pipeline wait that timed out) are recorded in a
- *    per-device error word.  Read it with fp8g_get_device_error().
+ *    per-device error word.  Read it with fp8g_get_device_error().  After a
+ *    timeout the outputs of the calls since the word was last cleared are
+ *    undefined (some CTAs gave up part-way).
  *  - The calls are thread-safe with respect to one another.
  *  - Needs a compute capability 10.0 device (B200); otherwise
  *    FP8G_ERR_UNSUPPORTED.
@@ -125,8 +128,9 @@ int m_grouped_fp8_gemm_nt_masked(const uint8_t *A, const float *sa, int ld_sa,
  *
  * Same operation, layouts, requirements and errors as fp8_gemm_nt.  It exists
  * for callers that must not call cudaMalloc when they run a GEMM: an engine
- * that hands out all device memory from its own pool, or code that runs while
- * a CUDA graph is being captured.  fp8_gemm_nt allocates a split-K workspace
+ * that hands out all device memory from its own pool, or a runtime that
+ * forbids allocation after start-up so that its footprint is fixed in
+ * advance.  fp8_gemm_nt allocates a split-K workspace
  * (about 4.7 MB) on the first decode-shaped call of each device; this entry
  * point instead keeps its scratch (the split-K partial sums and two counters
  * per tile) in a fixed array of 5 MiB + 1.25 KiB inside the library, which
@@ -143,10 +147,33 @@ int m_grouped_fp8_gemm_nt_masked(const uint8_t *A, const float *sa, int ld_sa,
  *  - All calls share the one array: calls whose executions overlap on the
  *    GPU (on different streams, or on one stream without ordering between
  *    them) race on it and give wrong results.  Order such calls.
+ *  - The CTAs of one tile add their partial sums inside the kernel, so they
+ *    must all be resident at once.  On a GPU shared with other work that may
+ *    not happen within the wait limit (1 s); the call then records
+ *    FP8G_DEVERR_TIMEOUT and D is undefined.
  */
 int fp8_gemm_nt_no_alloc(const uint8_t *A, const float *sa, int ld_sa,
                          const uint8_t *B, const float *sb,
                          uint16_t *D, int M, int N, int K, cudaStream_t stream);
+
+/*
+ * Host helper: converts A's scales from the row-major layout a quantiser
+ * naturally produces, src[g][m][kb] (one row of KB scales per row of A), to
+ * the library's MN-major layout, dst[g][kb][ld_sa] (dst[(g*KB + kb)*ld_sa + m]
+ * = src[(g*rows + m)*KB + kb]).  Entries m in [rows, ld_sa) of dst are set to
+ * zero.  The pages leave the scale layout open; they only say that the
+ * fine-grained scales come with the inputs (GeekNews, "DeepSeek, DeepGEMM
+ * 오픈소스 공개", topic body, first bullet) and that preparing inputs is the
+ * caller's job (kakushin.no, "Hvorfor FP8 og FP4 er interessant").
+ *   src, dst: HOST pointers owned by the caller, not overlapping;
+ *             src holds G*rows*KB floats, dst G*KB*ld_sa floats.
+ *   G >= 1 groups (1 for dense and contiguous, G for the masked layout),
+ *   rows >= 0 (M, or Mmax for masked), KB = K/128 >= 1,
+ *   ld_sa >= rows and ld_sa % 4 == 0 (the GEMM calls' requirement).
+ * Returns FP8G_OK; FP8G_ERR_INVALID_ARG for a null pointer or a bad size,
+ * FP8G_ERR_MISALIGNED if ld_sa % 4 != 0.  Touches no device and no CUDA API.
+ */
+int fp8g_sa_to_mn_major(const float *src, float *dst, int G, int rows, int KB, int ld_sa);
 
 /* Human-readable name of a status code (static string). */
 const char *fp8g_status_string(int status);

@@ -123,3 +123,33 @@ def test_every_variant_name_starts_with_its_kind(lib):
         assert n.split("_", 1)[0] in ("dense", "contiguous", "masked"), n
     for kind in ("dense", "contiguous", "masked"):
         assert any(n.startswith(kind + "_") for n in names), kind
+
+
+def test_sa_to_mn_major_round_trips_ragged_rows(lib):
+    """The host helper turns [G][rows][KB] scales into the library's
+    [G][KB][ld_sa] layout: checked against the generator's MN-major output
+    for a ragged row count (dense) and a grouped (masked) layout."""
+    import numpy as np
+    from fp8_block_scaled_x128_b200 import synth
+    f = lib.fp8g_sa_to_mn_major
+    f.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int]
+    ptr = lambda a: a.ctypes.data_as(C.c_void_p)
+    # dense, M = 77 (not a multiple of 4), K = 640
+    _, sa = synth.make_a(3, 77, 640)              # [KB][ld_sa], zero beyond row 77
+    KB, ld = sa.shape
+    rows_major = np.ascontiguousarray(sa[:, :77].T)  # [M][KB], what a row-wise quantiser yields
+    out = np.full((KB, ld), np.nan, np.float32)
+    assert f(ptr(rows_major), ptr(out), 1, 77, KB, ld) == 0
+    assert np.array_equal(out, sa)
+    # grouped: [G][Mmax][KB] -> [G][KB][ld_sa]
+    d = synth.masked_inputs(4, 3, 37, 8, 384)
+    src = np.ascontiguousarray(np.transpose(d["sa"][:, :, :37], (0, 2, 1)))
+    out = np.full(d["sa"].shape, np.nan, np.float32)
+    assert f(ptr(src), ptr(out), 3, 37, 3, d["ld_sa"]) == 0
+    assert np.array_equal(out, d["sa"])
+    # argument checks
+    assert f(None, ptr(out), 1, 4, 3, 4) == 1
+    assert f(ptr(src), ptr(out), 0, 4, 3, 4) == 1       # G < 1
+    assert f(ptr(src), ptr(out), 1, 8, 3, 4) == 1       # ld_sa < rows
+    assert f(ptr(src), ptr(out), 1, 4, 0, 4) == 1       # KB < 1
+    assert f(ptr(src), ptr(out), 1, 5, 3, 6) == 2       # ld_sa % 4 != 0

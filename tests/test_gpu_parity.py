@@ -265,14 +265,33 @@ def test_masked_in_cuda_graph_reads_counts_on_device(g):
 
 # --------------------------------------------------------------------------- full-size configurations
 
+def outlier_rows(seed, M, K, frac):
+    """Rows of A holding at least one x50 group, read from the generator's own
+    outlier stream (the same draw make_a uses), not from the oracle."""
+    KB = K // 128
+    u = synth.uniform(synth.stream_key(seed, synth.STREAM_OUTLIER), 0, M * KB).reshape(M, KB)
+    return np.nonzero((u < frac).any(axis=1))[0].astype(np.int32)
+
+
 @pytest.mark.slow
 def test_config_dense_4096x7168x16384_sampled_rows(g):
-    d = synth.config_inputs("dense_4096x7168x16384")
+    name = "dense_4096x7168x16384"
+    d = synth.config_inputs(name)
     got = dense_gpu(g, d)
     rng = np.random.default_rng(0)
+    # a random row subsample, compared on all N columns
     rows = np.unique(np.r_[0, 4095, 127, 128, rng.choice(4096, 44, replace=False)]).astype(np.int32)
     ex, _ = oracle_dense(d, rows=rows)
-    assert_close(got[rows], ex, "dense_4096x7168x16384 sampled")
+    assert_close(got[rows], ex, f"{name} sampled rows")
+    # every row that holds a x50 group, on one 128-column block of B (the
+    # oracle computes those columns from that block's rows of B and sb)
+    orows = outlier_rows(0, d["M"], d["K"], synth.CONFIGS[name]["outlier_frac"])
+    assert 0.6 * d["M"] < len(orows) < 0.85 * d["M"]  # 1 - 0.99^128 of the rows
+    for nb in (int(rng.integers(0, d["N"] // 128)), d["N"] // 128 - 1):
+        cols = slice(128 * nb, 128 * nb + 128)
+        ex, _ = oracle.gemm_nt(d["A"], d["sa"], d["ld_sa"], d["B"][cols], d["sb"][nb:nb + 1], d["M"], 128,
+                               d["K"], rows=orows)
+        assert_close(got[orows, cols], ex, f"{name} outlier rows, columns {cols}")
 
 
 @pytest.mark.slow
@@ -291,19 +310,14 @@ def test_config_contiguous_sampled_rows(g):
 
 
 @pytest.mark.slow
-def test_config_masked_sampled_rows(g):
+def test_config_masked_in_full(g):
     d = synth.config_inputs("masked_g16_m256_n4096_k7168")
     got = masked_gpu(g, d, expected_m=d["expected_m"])
     G, Mmax, N, K = d["G"], d["Mmax"], d["N"], d["K"]
-    mm = d["masked_m"]
+    mm = np.minimum(d["masked_m"], Mmax)
     live = np.arange(Mmax)[None, :] < mm[:, None]
     assert np.all(got[~live] == CANARY)
-    rng = np.random.default_rng(2)
+    ex, _ = oracle.m_grouped_masked(d["A"], d["sa"], d["ld_sa"], d["B"], d["sb"], d["masked_m"], G, Mmax, N, K)
     for gi in range(G):
-        if mm[gi] == 0:
-            continue
-        rows = np.unique(np.r_[0, mm[gi] - 1, rng.choice(mm[gi], min(6, mm[gi]), replace=False)]).astype(np.int32)
-        # one group's masked rows are that group's dense product (pinned in the oracle tests)
-        ex, _ = oracle.gemm_nt(d["A"][gi], d["sa"][gi], d["ld_sa"], d["B"][gi], d["sb"][gi], Mmax, N, K,
-                               rows=rows)
-        assert_close(got[gi][rows], ex, f"masked group {gi}")
+        assert_close(got[gi][:mm[gi]], ex[gi][:mm[gi]], f"masked group {gi} ({mm[gi]} rows)")
+    assert g.device_error() == 0

@@ -1,9 +1,12 @@
 """The dense entry point that allocates no device memory, on the GPU.
 
-fp8_gemm_nt_no_alloc is for callers that cannot allocate device memory when
-they run a GEMM (a fixed memory pool, or code running during graph capture):
-its split-K scratch is a fixed array inside the library instead of a
-workspace allocated on first use.  This file is collected last so that a run
+fp8_gemm_nt_no_alloc serves callers that cannot allocate device memory when
+they run a GEMM: an engine that hands out all memory from its own fixed pool,
+or a runtime that forbids allocation after start-up.  Its split-K scratch is a
+fixed array inside the library instead of a workspace allocated on first use.
+The outputs are checked against the CPU oracle (and bit for bit on
+exact-integer inputs) on two calls in a row, the second reusing the scratch
+the first one left behind.  This file is collected last so that a run
 stopping at the first failure has already run every other test; it passes
 both on its own in a fresh process and after the other tests.
 """
@@ -11,9 +14,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from fp8_block_scaled_x128_b200 import synth
 
-from .parity_util import assert_close, bf16_to_f64
+from .parity_util import assert_close, exact_integer_codes, pow2_scales
 
 pytestmark = pytest.mark.gpu
 
@@ -23,6 +27,7 @@ def g():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     from fp8_block_scaled_x128_b200 import gemm
+    gemm.device_error(clear=True)
     yield gemm
     gemm.set_variant_override(None)
 
@@ -36,19 +41,40 @@ def _bits(t):
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("shape", [(64, 2112, 7168), (1, 8, 128), (65, 520, 1024)],
-                         ids=lambda s: "x".join(map(str, s)))
-def test_no_alloc_matches_regular_entry_point_on_two_calls(g, shape):
-    M, N, K = shape
-    d = synth.dense_inputs(77 + M, M, N, K)
+def _two_calls(g, d):
     t = _dev(d)
-    ref = _bits(g.fp8_gemm_nt(t["A"], t["sa"], t["B"], t["sb"]))
-    D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    for call in range(2):  # the second call reuses the scratch the first one left behind
+    D = torch.empty((d["M"], d["N"]), dtype=torch.bfloat16, device="cuda")
+    out = []
+    for _ in range(2):
         D.view(torch.int16).fill_(0x7F7F)
         g.fp8_gemm_nt_no_alloc(t["A"], t["sa"], t["B"], t["sb"], D=D)
-        got = _bits(D)
-        assert_close(got, bf16_to_f64(ref), f"no-alloc call {call} {shape}")
+        out.append(_bits(D))
+    return out
+
+
+@pytest.mark.parametrize("shape", [(64, 2112, 7168), (1, 8, 128), (65, 520, 1024)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_no_alloc_matches_oracle_on_two_calls(g, shape):
+    M, N, K = shape
+    d = synth.dense_inputs(77 + M, M, N, K)
+    ex, _ = oracle.gemm_nt(d["A"], d["sa"], d["ld_sa"], d["B"], d["sb"], M, N, K)
+    for call, got in enumerate(_two_calls(g, d)):
+        assert_close(got, ex, f"no-alloc call {call} {shape}")
+    assert g.device_error() == 0
+
+
+def test_no_alloc_exact_integers_bit_exact_on_two_calls(g):
+    M, N, K = 64, 1040, 2048
+    rng = np.random.default_rng(11)
+    KB, NB = K // 128, (N + 127) // 128
+    ld = synth.ld_for(M)
+    sa = np.zeros((KB, ld), np.float32)
+    sa[:, :M] = pow2_scales(rng, (KB, M))
+    d = dict(A=exact_integer_codes(rng, (M, K)), sa=sa, ld_sa=ld, B=exact_integer_codes(rng, (N, K)),
+             sb=pow2_scales(rng, (NB, KB)), M=M, N=N, K=K)
+    _, bf = oracle.gemm_nt(d["A"], d["sa"], ld, d["B"], d["sb"], M, N, K)
+    for got in _two_calls(g, d):
+        assert np.array_equal(got, bf)
     assert g.device_error() == 0
 
 
