@@ -35,17 +35,17 @@ struct Variant {
   int launch_regs;  // register-split variants: registers per thread at launch
 };
 
-template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT>
+template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int OPT = 0>
 Variant make_variant(const char* name) {
   using L = Layout<kSwap, BNC, STAGES, SPLIT>;
   return Variant{name, KIND, kSwap, BNC, STAGES, SPLIT, L::kRegSplit,
-                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT>, L::kSmemAlloc, false,
+                 &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT, OPT>, L::kSmemAlloc, false,
                  kThreads, kLaunchRegs};
 }
 
-template <int KIND, int STAGES, int BN>
+template <int KIND, int STAGES, int BN, int OPT = 0>
 Variant make_pair_variant(const char* name) {
-  return Variant{name, KIND, false, BN, STAGES, 1, PairShape<BN>::kRegSplit, &fp8_gemm_pair_kernel<KIND, STAGES, BN>,
+  return Variant{name, KIND, false, BN, STAGES, 1, PairShape<BN>::kRegSplit, &fp8_gemm_pair_kernel<KIND, STAGES, BN, OPT>,
                  PairLayout<STAGES, BN>::kSmemAlloc, true, PairShape<BN>::kThreads, PairShape<BN>::kLaunchRegs};
 }
 
@@ -68,6 +68,13 @@ const Variant kVariants[] = {
     make_variant<false, 128, 6, kMasked, 1>("masked_mlanes_bn128_st6"),
     make_variant<false, 256, 4, kMasked, 1>("masked_mlanes_bn256_st4"),
     make_pair_variant<kMasked, 6, 192>("masked_mlanes_pair_bn192_st6"),
+    // promotion experiments (e = early release, f = packed FP32x2 FMA)
+    make_pair_variant<kDense, 8, 192, kOptEarly>("dense_mlanes_pair_bn192_st8_e"),
+    make_pair_variant<kDense, 8, 192, kOptEarly | kOptFma2>("dense_mlanes_pair_bn192_st8_ef"),
+    make_pair_variant<kDense, 8, 192, kOptFma2>("dense_mlanes_pair_bn192_st8_f"),
+    make_pair_variant<kContiguous, 8, 192, kOptEarly | kOptFma2>("contiguous_mlanes_pair_bn192_st8_ef"),
+    make_variant<false, 256, 4, kContiguous, 1, kOptFma2>("contiguous_mlanes_bn256_st4_f"),
+    make_pair_variant<kMasked, 6, 192, kOptEarly | kOptFma2>("masked_mlanes_pair_bn192_st6_ef"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
@@ -85,6 +92,12 @@ enum : int {
   V_MASKED_M128,
   V_MASKED_M256,
   V_MASKED_PAIR192,
+  V_X_DENSE_PAIR_E,
+  V_X_DENSE_PAIR_EF,
+  V_X_DENSE_PAIR_F,
+  V_X_CONTIG_PAIR_EF,
+  V_X_CONTIG_M256_F,
+  V_X_MASKED_PAIR_EF,
   V_COUNT
 };
 static_assert(V_COUNT == kNumVariants, "variant table and names");

@@ -122,6 +122,14 @@ constexpr int kGlobalSplit = -1;
 constexpr int kGlobalSplitPartials = -2;
 constexpr int kMaxGSplit = 16;  // the host never picks more
 
+// OPT bits of the promotion (template parameter of both kernels):
+//   kOptEarly: load all of a warp's columns of the partial from TMEM, release
+//              the buffer, then multiply-add (the MMA of K-block k + 2 waits
+//              only for the loads of k, not for its arithmetic; CTA-pair
+//              kernel only);
+//   kOptFma2:  packed FP32x2 fused multiply-adds (each half rounds like fmaf).
+constexpr int kOptEarly = 1, kOptFma2 = 2;
+
 constexpr int pow2_at_least(int x, int lo) {
   int p = lo;
   while (p < x) p *= 2;
@@ -323,7 +331,7 @@ __device__ __forceinline__ void global_split_reduce(const Params& p, int tile, u
   }
 }
 
-template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT>
+template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int OPT = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSA, const Params p) {
@@ -543,8 +551,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int j = 0; j < kGroup; ++j) {
                 float* a = acc + 32 * (j0 + j);
+                if constexpr ((OPT & kOptFma2) != 0) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
+                  for (int c = 0; c < 32; c += 2) ffma2(a[c], a[c + 1], r[j][c], r[j][c + 1], sc2[u]);
+                } else {
+#pragma unroll
+                  for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
+                }
               }
             }
             tc_fence_before();

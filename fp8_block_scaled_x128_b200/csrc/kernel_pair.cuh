@@ -145,7 +145,8 @@ __device__ __forceinline__ PairTile get_pair_tile(const Params& p, int t, int ps
   return T;
 }
 
-template <int KIND, int STAGES, int BN = 256>
+// OPT: promotion options (kOptEarly, kOptFma2; kernel.cuh).
+template <int KIND, int STAGES, int BN = 256, int OPT = 0>
 __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmSA, const Params p) {
@@ -329,6 +330,38 @@ __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
           tc_fence_after();
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
                                  static_cast<uint32_t>(b * BNC + wg * kCW);
+          if constexpr ((OPT & kOptEarly) != 0) {
+            // every column of this warp's partial into registers, then the
+            // buffer goes back to the MMA before the arithmetic
+            constexpr int kCh = kCW / 32;
+            uint32_t r[kCh][32];
+            if (T.active) {
+#pragma unroll
+              for (int j = 0; j < kCh; ++j) tmem_ld_32x32b_x32(taddr + 32 * j, r[j]);
+              tmem_ld_wait_bind(r[0]);
+#pragma unroll
+              for (int j = 1; j < kCh; ++j) bind_after_wait(r[j]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if (rank == 0) mbar_arrive_relaxed(tempty_bar(b));
+              else mbar_arrive_remote_relaxed(tempty_remote + 8u * b);
+            }
+            if (T.active) {
+#pragma unroll
+              for (int j = 0; j < kCh; ++j) {
+                float* a = acc + 32 * j;
+                if constexpr ((OPT & kOptFma2) != 0) {
+#pragma unroll
+                  for (int c = 0; c < 32; c += 2) ffma2(a[c], a[c + 1], r[j][c], r[j][c + 1], sc2[u]);
+                } else {
+#pragma unroll
+                  for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
+                }
+              }
+            }
+          } else {
           constexpr int kG = S::kGroup;
           // a CTA whose block belongs to the other expert of this pass only
           // hands the buffer back
@@ -344,8 +377,13 @@ __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
 #pragma unroll
               for (int j = 0; j < kG; ++j) {
                 float* a = acc + 32 * (j0 + j);
+                if constexpr ((OPT & kOptFma2) != 0) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
+                  for (int c = 0; c < 32; c += 2) ffma2(a[c], a[c + 1], r[j][c], r[j][c + 1], sc2[u]);
+                } else {
+#pragma unroll
+                  for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
+                }
               }
             }
           }
@@ -354,6 +392,7 @@ __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
           if (lane == 0) {
             if (rank == 0) mbar_arrive_relaxed(tempty_bar(b));
             else mbar_arrive_remote_relaxed(tempty_remote + 8u * b);
+          }
           }
           ++it;
         }

@@ -306,6 +306,20 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N) {
   return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// a0 += p0 * s, a1 += p1 * s as one packed FP32x2 fused multiply-add
+// (fma.rn.f32x2, sm_100): each half rounds exactly like fmaf, at half the
+// instruction count.  p0, p1 are raw FP32 bit patterns (from tcgen05.ld).
+__device__ __forceinline__ void ffma2(float& a0, float& a1, uint32_t p0, uint32_t p1, float s) {
+  asm("{\n\t.reg .b64 acc, prt, scl;\n\t"
+      "mov.b64 acc, {%0, %1};\n\t"
+      "mov.b64 prt, {%2, %3};\n\t"
+      "mov.b64 scl, {%4, %4};\n\t"
+      "fma.rn.f32x2 acc, prt, scl, acc;\n\t"
+      "mov.b64 {%0, %1}, acc;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(p0), "r"(p1), "f"(s));
+}
+
 // FP32 pair -> packed bf16x2, round to nearest even (lo in the low half).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -33,6 +33,12 @@ def load(path: str):
     L.fp8o_m_grouped_contiguous.argtypes = [P, P, i, P, P, P, i, i, i, i, P, i, P, P, i]
     L.fp8o_m_grouped_masked.restype = i
     L.fp8o_m_grouped_masked.argtypes = [P, P, i, P, P, P, i, i, i, i, P, P, i]
+    L.fp8o_e4m3_encode.restype = C.c_uint8
+    L.fp8o_e4m3_encode.argtypes = [C.c_float]
+    L.fp8o_quantize_1x128.restype = i
+    L.fp8o_quantize_1x128.argtypes = [P, i, i, P, P, i]
+    L.fp8o_quantize_128x128.restype = i
+    L.fp8o_quantize_128x128.argtypes = [P, i, i, P, P]
     return L
 
 
@@ -122,3 +128,31 @@ def m_grouped_masked(A, sa, ld_sa, B, sb, masked_m, G, Mmax, N, K, nthreads=None
     if rc:
         raise ValueError("oracle: bad arguments")
     return ex, bf
+
+
+def e4m3_encode(x: float) -> int:
+    return lib().fp8o_e4m3_encode(float(x))
+
+
+def quantize_1x128(x, ld_sa=None):
+    """Activations x [rows, K] (float32; bf16 values converted exactly) ->
+    (codes uint8 [rows, K], sa float32 [KB, ld_sa]; entries past rows are 0)."""
+    x = _c(x, np.float32)
+    rows, K = x.shape
+    ld = max(4, (rows + 3) // 4 * 4) if ld_sa is None else int(ld_sa)
+    q = np.zeros((rows, K), np.uint8)
+    sa = np.zeros((K // 128 if K % 128 == 0 else 1, ld), np.float32)
+    if lib().fp8o_quantize_1x128(_p(x), int(rows), int(K), _p(q), _p(sa), int(ld)):
+        raise ValueError("oracle: bad arguments")
+    return q, sa
+
+
+def quantize_128x128(x):
+    """Weights x [N, K] float32 -> (codes uint8 [N, K], sb float32 [NB, KB])."""
+    x = _c(x, np.float32)
+    N, K = x.shape
+    q = np.zeros((N, K), np.uint8)
+    sb = np.zeros(((N + 127) // 128, max(1, K // 128)), np.float32)
+    if lib().fp8o_quantize_128x128(_p(x), int(N), int(K), _p(q), _p(sb)):
+        raise ValueError("oracle: bad arguments")
+    return q, sb

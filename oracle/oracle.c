@@ -297,3 +297,105 @@ int fp8o_m_grouped_masked(const uint8_t *A, const float *sa, int ld_sa,
     free(tasks);
     return 0;
 }
+
+/* ===========================================================================
+ * FP8 quantisation of the GEMM's inputs.  The pages leave this step to the
+ * user (kakushin.no, "Hvorfor FP8 og FP4 er interessant": inputs must be
+ * converted to FP8 by the caller); the granularity is the one of the GEMM
+ * above (one FP32 scale per 1x128 row group of A, per 128x128 block of B).
+ * Readings, since the pages give no formula: scale = amax / 448 in FP32 (448
+ * is the largest finite e4m3 value), scale = 1 for an all-zero group, and
+ * code = e4m3_rne_satfinite(x / scale) with x / scale one IEEE FP32 division.
+ * These functions work in FP32 because that is the precision in which the
+ * scale and the quotient are defined; the e4m3 rounding itself is done
+ * exactly (in double) from the format definition.
+ * ======================================================================== */
+
+/* e4m3 ("fn") code of a finite float: round to nearest, ties to even, values
+ * beyond the largest finite magnitude (448) saturate to +-448; the sign of
+ * zero is kept.  Normal codes: (1 + m/8) * 2^(e-7), e = 1..15 (e = 15 only up
+ * to m = 6); subnormals: (m/8) * 2^-6.  */
+uint8_t fp8o_e4m3_encode(float x)
+{
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    int E, e;
+    double q, steps;
+    if (a == 0.0)
+        return sign;
+    (void)frexp(a, &E);        /* a = f * 2^E, f in [0.5, 1) */
+    e = E - 1;                 /* a in [2^e, 2^(e+1)) */
+    if (e < -6)
+        e = -6;                /* subnormals share the quantum 2^-9 */
+    q = ldexp(1.0, e - 3);     /* 3 mantissa bits */
+    steps = nearbyint(a / q);  /* exact quotient; ties to even */
+    if (steps >= 16.0) {       /* mantissa carried into the exponent */
+        steps = 8.0;
+        e += 1;
+    }
+    if (e > 8 || (e == 8 && steps > 14.0))
+        return sign | 0x7E;    /* saturate to 448 = 1.75 * 2^8 */
+    if (steps < 8.0)           /* subnormal (only at e == -6) */
+        return sign | (uint8_t)steps;
+    return sign | (uint8_t)(((e + 7) << 3) | ((int)steps - 8));
+}
+
+static float scale_of_amax(float amax)
+{
+    return amax > 0.0f ? amax / 448.0f : 1.0f;
+}
+
+/* Activations: x [rows][K] (K % 128 == 0) -> q [rows][K] e4m3 codes and
+ * sa [KB][ld_sa] (the GEMM's MN-major layout): one scale per 1x128 group of
+ * a row.  Entries of sa past `rows` are not written.  Returns 0, or -1 on a
+ * bad argument. */
+int fp8o_quantize_1x128(const float *x, int rows, int K, uint8_t *q, float *sa, int ld_sa)
+{
+    if (K <= 0 || K % 128 || rows < 0 || ld_sa < rows)
+        return -1;
+    int KB = K / 128;
+    for (long r = 0; r < rows; ++r) {
+        for (int kb = 0; kb < KB; ++kb) {
+            const float *g = x + r * K + (long)kb * 128;
+            float amax = 0.0f;
+            for (int j = 0; j < 128; ++j)
+                if (fabsf(g[j]) > amax)
+                    amax = fabsf(g[j]);
+            float s = scale_of_amax(amax);
+            for (int j = 0; j < 128; ++j)
+                q[r * K + (long)kb * 128 + j] = fp8o_e4m3_encode(g[j] / s);
+            sa[(long)kb * ld_sa + r] = s;
+        }
+    }
+    return 0;
+}
+
+/* Weights: x [N][K] (K % 128 == 0) -> q [N][K] codes and sb [NB][KB]: one
+ * scale per 128x128 block; the last block row holds the N % 128 remaining
+ * rows when N is not a multiple of 128.  Returns 0, or -1 on a bad argument. */
+int fp8o_quantize_128x128(const float *x, int N, int K, uint8_t *q, float *sb)
+{
+    if (K <= 0 || K % 128 || N < 0)
+        return -1;
+    int KB = K / 128, NB = (N + 127) / 128;
+    for (int nb = 0; nb < NB; ++nb) {
+        int r0 = nb * 128, r1 = r0 + 128 < N ? r0 + 128 : N;
+        for (int kb = 0; kb < KB; ++kb) {
+            float amax = 0.0f;
+            for (long r = r0; r < r1; ++r)
+                for (int j = 0; j < 128; ++j) {
+                    float v = fabsf(x[r * K + (long)kb * 128 + j]);
+                    if (v > amax)
+                        amax = v;
+                }
+            float s = scale_of_amax(amax);
+            for (long r = r0; r < r1; ++r)
+                for (int j = 0; j < 128; ++j) {
+                    long i = r * K + (long)kb * 128 + j;
+                    q[i] = fp8o_e4m3_encode(x[i] / s);
+                }
+            sb[(long)nb * KB + kb] = s;
+        }
+    }
+    return 0;
+}

@@ -14,6 +14,7 @@ import oracle
 from oracle.build import SRC as ORACLE_SRC
 
 from . import test_oracle_pins as pins
+from . import test_oracle_quant_pins as qpins
 
 MUTANTS = {
     "decode_bias": ("v = ldexp(8.0 + (double)m, e - 7 - 3);", "v = ldexp(8.0 + (double)m, e - 8 - 3);"),
@@ -31,6 +32,17 @@ MUTANTS = {
     "contig_no_skip": ("if (g < 0)\n            continue;", "if (g < 0)\n            g = 0;"),
     "masked_row_shift": ("long orow = (long)g * Mmax + m;", "long orow = (long)g * Mmax + (m + 1 < Mmax ? m + 1 : m);"),
     "masked_group_sa": ("sa + (long)g * KB * ld_sa + m", "sa + m"),
+    # the FP8 quantiser
+    "enc_truncates": ("steps = nearbyint(a / q);", "steps = floor(a / q);"),
+    "enc_ties_away": ("steps = nearbyint(a / q);", "steps = round(a / q);"),
+    "enc_no_saturation": ("return sign | 0x7E;    /* saturate", "return sign | 0x7F;    /* saturate"),
+    "enc_subnormal_quantum": ("if (e < -6)\n        e = -6;", "if (e < -7)\n        e = -7;"),
+    "quant_scale_divisor": ("return amax > 0.0f ? amax / 448.0f : 1.0f;", "return amax > 0.0f ? amax / 240.0f : 1.0f;"),
+    "quant_group_width": ("for (int j = 0; j < 128; ++j)\n                if (fabsf(g[j]) > amax)",
+                          "for (int j = 0; j < 64; ++j)\n                if (fabsf(g[j]) > amax)"),
+    "quant_sa_layout": ("sa[(long)kb * ld_sa + r] = s;", "sa[r * KB + kb] = s;"),
+    "quant_block_rows": ("for (long r = r0; r < r1; ++r)\n                for (int j = 0; j < 128; ++j) {\n                    float v",
+                         "for (long r = r0; r < r0 + 1; ++r)\n                for (int j = 0; j < 128; ++j) {\n                    float v"),
 }
 
 # every pin that takes no parameters, plus the parametrised ones at one or two points
@@ -51,6 +63,13 @@ PINS = [
     pins.test_contiguous_padding_rows_do_not_affect_other_rows,
     pins.test_masked_rows_beyond_mask_untouched_and_valid_rows_match_bruteforce,
     pins.test_masked_group_permutation_and_independence,
+    qpins.test_encode_round_trips_every_finite_code,
+    qpins.test_encode_midpoints_round_to_even_and_saturate,
+    qpins.test_encode_matches_torch_and_the_generator_on_random_floats,
+    lambda: qpins.test_quantize_1x128_against_torch(37, 384),
+    qpins.test_quantize_1x128_error_bound_and_locality,
+    lambda: qpins.test_quantize_128x128_against_torch(200, 384),
+    qpins.test_quantize_128x128_block_is_shared_by_its_rows_only,
 ]
 
 
