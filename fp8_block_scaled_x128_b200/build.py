@@ -27,7 +27,7 @@ FLAGS = [
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + [os.path.join(INCLUDE, "fp8gemm.h"), __file__])
+                  + glob.glob(os.path.join(INCLUDE, "*.h")) + [__file__])
 
 
 def up_to_date() -> bool:

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "fp8gemm.h"
+#include "fp8gemm_testing.h"
 #include "kernel.cuh"
 #include "kernel_pair.cuh"
 
@@ -43,10 +44,11 @@ Variant make_variant(const char* name) {
                  kThreads, kLaunchRegs};
 }
 
-template <int KIND, int STAGES, int BN, int OPT = 0>
+template <int KIND, int STAGES, int BN, int OPT = 0, int NWG = default_nwg(BN)>
 Variant make_pair_variant(const char* name) {
-  return Variant{name, KIND, false, BN, STAGES, 1, PairShape<BN>::kRegSplit, &fp8_gemm_pair_kernel<KIND, STAGES, BN, OPT>,
-                 PairLayout<STAGES, BN>::kSmemAlloc, true, PairShape<BN>::kThreads, PairShape<BN>::kLaunchRegs};
+  using S = PairShape<BN, NWG>;
+  return Variant{name, KIND, false, BN, STAGES, 1, S::kRegSplit, &fp8_gemm_pair_kernel<KIND, STAGES, BN, OPT, NWG>,
+                 PairLayout<STAGES, BN>::kSmemAlloc, true, S::kThreads, S::kLaunchRegs};
 }
 
 // "nlanes": TMEM lanes are rows of B (small M); "mlanes": lanes are rows of A.
@@ -62,19 +64,12 @@ const Variant kVariants[] = {
     make_variant<true, 64, 8, kDense, kGlobalSplitPartials>("dense_nlanes_bn64_st8_gsplit_2k"),
     make_variant<false, 128, 6, kDense, 1>("dense_mlanes_bn128_st6"),
     make_variant<false, 256, 4, kDense, 1>("dense_mlanes_bn256_st4"),
-    make_pair_variant<kDense, 8, 192>("dense_mlanes_pair_bn192_st8"),
+    make_pair_variant<kDense, 8, 192, kOptFma2>("dense_mlanes_pair_bn192_st8_f"),
     make_variant<false, 128, 6, kContiguous, 1>("contiguous_mlanes_bn128_st6"),
     make_variant<false, 256, 4, kContiguous, 1>("contiguous_mlanes_bn256_st4"),
     make_variant<false, 128, 6, kMasked, 1>("masked_mlanes_bn128_st6"),
     make_variant<false, 256, 4, kMasked, 1>("masked_mlanes_bn256_st4"),
     make_pair_variant<kMasked, 6, 192>("masked_mlanes_pair_bn192_st6"),
-    // promotion experiments (e = early release, f = packed FP32x2 FMA)
-    make_pair_variant<kDense, 8, 192, kOptEarly>("dense_mlanes_pair_bn192_st8_e"),
-    make_pair_variant<kDense, 8, 192, kOptEarly | kOptFma2>("dense_mlanes_pair_bn192_st8_ef"),
-    make_pair_variant<kDense, 8, 192, kOptFma2>("dense_mlanes_pair_bn192_st8_f"),
-    make_pair_variant<kContiguous, 8, 192, kOptEarly | kOptFma2>("contiguous_mlanes_pair_bn192_st8_ef"),
-    make_variant<false, 256, 4, kContiguous, 1, kOptFma2>("contiguous_mlanes_bn256_st4_f"),
-    make_pair_variant<kMasked, 6, 192, kOptEarly | kOptFma2>("masked_mlanes_pair_bn192_st6_ef"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
@@ -92,17 +87,15 @@ enum : int {
   V_MASKED_M128,
   V_MASKED_M256,
   V_MASKED_PAIR192,
-  V_X_DENSE_PAIR_E,
-  V_X_DENSE_PAIR_EF,
-  V_X_DENSE_PAIR_F,
-  V_X_CONTIG_PAIR_EF,
-  V_X_CONTIG_M256_F,
-  V_X_MASKED_PAIR_EF,
   V_COUNT
 };
 static_assert(V_COUNT == kNumVariants, "variant table and names");
 
 std::atomic<int> g_override{-1};
+
+// test hook (fp8g_testing_withhold_stage): -1 = off
+std::atomic<int> g_test_withhold{-1};
+std::atomic<uint32_t> g_test_wait_limit_us{kWaitLimitUs};
 
 // Programmatic dependent launch is on unless FP8G_DISABLE_PDL is set to a
 // nonzero value in the environment (read once).
@@ -330,6 +323,10 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   p.ld_sa = P.ld_sa;
   p.sb = P.sb;
   p.D = P.D;
+  // the test hook applies to the single-CTA kernel only
+  const int withhold = V.pair ? -1 : g_test_withhold.load(std::memory_order_relaxed);
+  p.test_withhold_it = withhold;
+  p.wait_limit_us = withhold >= 0 ? g_test_wait_limit_us.load(std::memory_order_relaxed) : kWaitLimitUs;
   if (p.num_tiles <= 0) return FP8G_OK;
   if (V.split < 0) {
     p.gsplit = gsplit_for(dev, p.num_tiles, KB);
@@ -583,7 +580,19 @@ const char* fp8g_variant_name(int variant) {
 
 int fp8g_last_variant(void) { return t_last_variant; }
 
-int fp8g_version(void) { return 100; }
+int fp8g_version(void) { return 200; }
+
+int fp8g_testing_withhold_stage(int iteration, unsigned wait_limit_us) {
+  if (iteration < 0) {
+    g_test_withhold.store(-1, std::memory_order_relaxed);
+    g_test_wait_limit_us.store(kWaitLimitUs, std::memory_order_relaxed);
+    return FP8G_OK;
+  }
+  if (wait_limit_us < 100 || wait_limit_us > kWaitLimitUs) return FP8G_ERR_INVALID_ARG;
+  g_test_wait_limit_us.store(wait_limit_us, std::memory_order_relaxed);
+  g_test_withhold.store(iteration, std::memory_order_relaxed);
+  return FP8G_OK;
+}
 
 }  // extern "C"
 
@@ -671,6 +680,8 @@ extern "C" int fp8_gemm_nt_no_alloc(const uint8_t* A, const float* sa, int ld_sa
   p.sb = sb;
   p.D = D;
   p.gsplit = gsplit;
+  p.wait_limit_us = kWaitLimitUs;
+  p.test_withhold_it = -1;
   p.ws = static_cast<float*>(scratch);
   p.sync = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(scratch) + kNoAllocPartialBytes);
   // the counters of this call start at zero even if an earlier call gave up

@@ -87,7 +87,7 @@ constexpr int kThreads = 384;
 constexpr int kIssuersPerWarp = 4;                  // TMA-issuing lanes in each producer warp
 constexpr int kIssuers = 2 * kIssuersPerWarp;       // warps 0 and 3
 constexpr int kKBMax = 512;                         // K <= 65536
-constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s
+constexpr uint32_t kWaitLimitUs = 1000000u;         // 1 s: the default wait limit
 constexpr uint64_t kDrainTimeoutNs = 100000000ull;  // 0.1 s
 
 // Per-device error word (FP8G_DEVERR_* bits); read by fp8g_get_device_error.
@@ -112,6 +112,12 @@ struct Params {
   int gsplit;
   float* ws;
   uint32_t* sync;
+  // every pipeline wait gives up after wait_limit_us microseconds; a test
+  // hook may also make the TMA producers of the single-CTA kernel skip the
+  // loads of pipeline iteration test_withhold_it (-1: none), so that a wait
+  // runs out without any fault
+  uint32_t wait_limit_us;
+  int test_withhold_it;
 };
 
 // SPLIT template values selecting the global-memory split-K (count at run
@@ -123,12 +129,12 @@ constexpr int kGlobalSplitPartials = -2;
 constexpr int kMaxGSplit = 16;  // the host never picks more
 
 // OPT bits of the promotion (template parameter of both kernels):
-//   kOptEarly: load all of a warp's columns of the partial from TMEM, release
-//              the buffer, then multiply-add (the MMA of K-block k + 2 waits
-//              only for the loads of k, not for its arithmetic; CTA-pair
-//              kernel only);
-//   kOptFma2:  packed FP32x2 fused multiply-adds (each half rounds like fmaf).
-constexpr int kOptEarly = 1, kOptFma2 = 2;
+//   kOptFma2: packed FP32x2 fused multiply-adds (fma.rn.f32x2; each half
+//             rounds like fmaf, so results are unchanged).  Measured on the
+//             large dense shape: 5-11 % fewer cycles on the CTA-pair kernel;
+//             slower on the single-CTA 256-wide kernel, whose promotion
+//             threads then spill.
+constexpr int kOptFma2 = 2;
 
 constexpr int pow2_at_least(int x, int lo) {
   int p = lo;
@@ -237,7 +243,9 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int t, uint32_t rank, 
 }
 
 // Bounded wait on a local mbarrier phase.  Returns false on timeout (after
-// recording it) or when another role has already aborted.
+// recording it) or when another role has already aborted.  ctl[0] is the
+// CTA's abort flag, ctl[1] the wait limit in microseconds (both in shared
+// memory, set up by thread 0 from Params::wait_limit_us).
 template <bool kClusterScope = false>
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
                                            volatile uint32_t* abort_flag) {
@@ -250,7 +258,8 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
     if (poll()) return true;
     if ((i & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      // the limit is read only here, off the path of a wait that completes
+      if (globaltimer_ns() - t0 > 1000ull * abort_flag[1]) {
         *abort_flag = 1u;
         atomicOr(&g_fp8g_error_word, FP8G_DEVERR_TIMEOUT);
         return false;
@@ -292,7 +301,7 @@ __device__ __forceinline__ void global_split_reduce(const Params& p, int tile, u
       const uint64_t t0 = globaltimer_ns();
       while (ld_acquire_gpu(arrive) < need) {
         if (*abort_flag) break;
-        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        if (globaltimer_ns() - t0 > 1000ull * abort_flag[1]) {
           *abort_flag = 1u;
           atomicOr(&g_fp8g_error_word, FP8G_DEVERR_TIMEOUT);
           break;
@@ -351,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + L::kNBuf + b); };
   auto drain_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + 2 * L::kNBuf + i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
-  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* abort_flag = tmem_slot + 1;  // [0] abort flag, [1] wait limit (us)
 
   // stage buffers
   auto lane_tile = [&](int s) { return sbase + L::kOffLane + s * L::kLaneBytes; };
@@ -372,7 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(drain_bar(0), 1);
     mbar_init(drain_bar(1), 1);
-    *abort_flag = 0u;
+    abort_flag[0] = 0u;
+    abort_flag[1] = p.wait_limit_us;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -428,6 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          if (static_cast<int>(it) == p.test_withhold_it) continue;  // test hook: this stage never fills
           mbar_arrive_expect_tx(full_bar(s), kStageTx);
           if constexpr (kSwap) {
             tma_load_3d(lane_tile(s), &tmB, full_bar(s), kb * 128, T.n0, gb);

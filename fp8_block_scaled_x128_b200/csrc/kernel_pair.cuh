@@ -31,19 +31,25 @@
 
 namespace fp8g {
 
-// BN: columns of the pair tile (the MMA's N).  256: two promotion
-// warpgroups of 128 columns; 192: three of 64 columns (512 threads), which
-// spreads the FP32 promotion over more warps at the cost of a narrower tile;
-// 128: two of 64 columns and four TMEM buffers instead of two, so the MMA may
-// run up to three K-blocks ahead of the promotion.
-template <int BN>
+// BN: columns of the pair tile (the MMA's N); NWG: promotion warpgroups,
+// each owning BN / NWG columns.  256 / 2: 128 columns per thread (384
+// threads); 192 / 3: 64 columns (512 threads), which spreads the FP32
+// promotion over more warps at the cost of a narrower tile; 128 / 2: 64
+// columns and four TMEM buffers instead of two, so the MMA may run up to
+// three K-blocks ahead of the promotion.
+constexpr int default_nwg(int BN) { return BN == 192 ? 3 : 2; }
+
+template <int BN, int NWG = default_nwg(BN)>
 struct PairShape {
   static_assert(BN == 256 || BN == 192 || BN == 128, "pair tile width");
-  static constexpr int kNWG = BN == 192 ? 3 : 2;          // promotion warpgroups
+  static_assert(NWG == default_nwg(BN), "promotion warpgroups");
+  static constexpr int kNWG = NWG;                        // promotion warpgroups
   static constexpr int kCW = BN / kNWG;                   // columns per promotion thread
   static constexpr int kThreads = 128 * (1 + kNWG);
+  // registers per thread at launch (the compiler's cap for kThreads per SM)
+  // and after the setmaxnreg split between the control and promotion roles
   static constexpr int kLaunchRegs = kNWG == 2 ? 168 : 128;
-  static constexpr bool kRegSplit = kCW > 64 || kNWG == 3;  // setmaxnreg between the roles
+  static constexpr bool kRegSplit = kCW > 64 || kNWG >= 3;
   static constexpr int kControlRegs = 56;
   static constexpr int kPromoRegs = kNWG == 2 ? 224 : 152;
   static constexpr int kGroup = kCW >= 128 ? 2 : 1;       // 32-column TMEM loads per wait
@@ -145,13 +151,13 @@ __device__ __forceinline__ PairTile get_pair_tile(const Params& p, int t, int ps
   return T;
 }
 
-// OPT: promotion options (kOptEarly, kOptFma2; kernel.cuh).
-template <int KIND, int STAGES, int BN = 256, int OPT = 0>
-__global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
+// OPT: promotion options (kOptFma2; kernel.cuh).
+template <int KIND, int STAGES, int BN = 256, int OPT = 0, int NWG = default_nwg(BN)>
+__global__ void __launch_bounds__(PairShape<BN, NWG>::kThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmSA, const Params p) {
   using L = PairLayout<STAGES, BN>;
-  using S = PairShape<BN>;
+  using S = PairShape<BN, NWG>;
   constexpr int BNC = BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + L::kNBuf + b); };
   auto drain_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + 2 * L::kNBuf + i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
-  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* abort_flag = tmem_slot + 1;  // [0] abort flag, [1] wait limit (us)
   auto a_tile = [&](int s) { return sbase + L::kOffA + s * L::kTileBytes; };
   auto b_tile = [&](int s) { return sbase + L::kOffB + s * L::kBTileBytes; };
 
@@ -183,7 +189,8 @@ __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
     }
     mbar_init(drain_bar(0), 1);
     mbar_init(drain_bar(1), 1);
-    *abort_flag = 0u;
+    abort_flag[0] = 0u;
+    abort_flag[1] = p.wait_limit_us;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -330,38 +337,6 @@ __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
           tc_fence_after();
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
                                  static_cast<uint32_t>(b * BNC + wg * kCW);
-          if constexpr ((OPT & kOptEarly) != 0) {
-            // every column of this warp's partial into registers, then the
-            // buffer goes back to the MMA before the arithmetic
-            constexpr int kCh = kCW / 32;
-            uint32_t r[kCh][32];
-            if (T.active) {
-#pragma unroll
-              for (int j = 0; j < kCh; ++j) tmem_ld_32x32b_x32(taddr + 32 * j, r[j]);
-              tmem_ld_wait_bind(r[0]);
-#pragma unroll
-              for (int j = 1; j < kCh; ++j) bind_after_wait(r[j]);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-              if (rank == 0) mbar_arrive_relaxed(tempty_bar(b));
-              else mbar_arrive_remote_relaxed(tempty_remote + 8u * b);
-            }
-            if (T.active) {
-#pragma unroll
-              for (int j = 0; j < kCh; ++j) {
-                float* a = acc + 32 * j;
-                if constexpr ((OPT & kOptFma2) != 0) {
-#pragma unroll
-                  for (int c = 0; c < 32; c += 2) ffma2(a[c], a[c + 1], r[j][c], r[j][c + 1], sc2[u]);
-                } else {
-#pragma unroll
-                  for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
-                }
-              }
-            }
-          } else {
           constexpr int kG = S::kGroup;
           // a CTA whose block belongs to the other expert of this pass only
           // hands the buffer back
@@ -392,7 +367,6 @@ __global__ void __launch_bounds__(PairShape<BN>::kThreads, 1)
           if (lane == 0) {
             if (rank == 0) mbar_arrive_relaxed(tempty_bar(b));
             else mbar_arrive_remote_relaxed(tempty_remote + 8u * b);
-          }
           }
           ++it;
         }

@@ -32,6 +32,12 @@ lib.fp8_gemm_nt_no_alloc.restype = _I
 lib.fp8_gemm_nt_no_alloc.argtypes = [_P, _P, _I, _P, _P, _P, _I, _I, _I, _P]
 lib.fp8g_sa_to_mn_major.restype = _I
 lib.fp8g_sa_to_mn_major.argtypes = [_P, _P, _I, _I, _I, _I]
+lib.fp8g_quantize_1x128.restype = _I
+lib.fp8g_quantize_1x128.argtypes = [_P, _I, _I, _I, _P, _P, _I, _P]
+lib.fp8g_quantize_128x128.restype = _I
+lib.fp8g_quantize_128x128.argtypes = [_P, _I, _I, _I, _P, _P, _P]
+lib.fp8g_testing_withhold_stage.restype = _I
+lib.fp8g_testing_withhold_stage.argtypes = [_I, C.c_uint]
 lib.fp8g_status_string.restype = C.c_char_p
 lib.fp8g_status_string.argtypes = [_I]
 lib.fp8g_get_device_error.restype = _I
@@ -97,6 +103,14 @@ def variant_names():
 
 def set_variant_override(v: int | None) -> None:
     _check(lib.fp8g_set_variant_override(-1 if v is None else int(v)), "fp8g_set_variant_override")
+
+
+def testing_withhold_stage(iteration: int | None, wait_limit_us: int = 2000) -> None:
+    """Test hook (include/fp8gemm_testing.h): from the next call on, the
+    single-CTA kernels skip the loads of pipeline iteration `iteration` and
+    give up on any wait after `wait_limit_us`; None turns it off."""
+    _check(lib.fp8g_testing_withhold_stage(-1 if iteration is None else int(iteration), int(wait_limit_us)),
+           "fp8g_testing_withhold_stage")
 
 
 def last_variant() -> int:
@@ -201,3 +215,49 @@ def sa_to_mn_major(sa_rows, ld_sa=None):
     _check(lib.fp8g_sa_to_mn_major(src.ctypes.data_as(_P), dst.ctypes.data_as(_P), G, rows, KB, ld),
            "fp8g_sa_to_mn_major")
     return dst if grouped else dst[0]
+
+
+_IN_DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+
+
+def _quant_input(x):
+    if not x.is_cuda or x.dtype not in _IN_DTYPE or not x.is_contiguous() or x.dim() != 2:
+        raise TypeError(f"x: expected a contiguous 2-D CUDA tensor of bfloat16 or float32, got {x.dtype} "
+                        f"{tuple(x.shape)} on {x.device}")
+    return x
+
+
+def quantize_1x128(x, q=None, sa=None, ld_sa=None, stream=None):
+    """Activations x [rows, K] (bfloat16 or float32) -> (q [rows, K] uint8 e4m3
+    codes, sa [K/128, ld_sa] float32 scales, one per 1x128 group), the GEMM's
+    A-side inputs.  ld_sa defaults to rows rounded up to a multiple of 4."""
+    _quant_input(x)
+    rows, K = x.shape
+    ld = max(4, (rows + 3) // 4 * 4) if ld_sa is None else int(ld_sa)
+    if q is None:
+        q = torch.empty((rows, K), dtype=torch.uint8, device=x.device)
+    if sa is None:
+        sa = torch.zeros((max(1, K // 128), ld), dtype=torch.float32, device=x.device)
+    _dev(q, torch.uint8, "q"), _dev(sa, torch.float32, "sa")
+    dev = _one_device(x=x, q=q, sa=sa)
+    with torch.cuda.device(dev):
+        _check(lib.fp8g_quantize_1x128(_ptr(x), _IN_DTYPE[x.dtype], rows, K, _ptr(q), _ptr(sa), sa.shape[-1],
+                                       _stream(stream, dev)), "fp8g_quantize_1x128")
+    return q, sa
+
+
+def quantize_128x128(x, q=None, sb=None, stream=None):
+    """Weights x [N, K] (bfloat16 or float32) -> (q [N, K] uint8 e4m3 codes,
+    sb [ceil(N/128), K/128] float32 scales, one per 128x128 block)."""
+    _quant_input(x)
+    N, K = x.shape
+    if q is None:
+        q = torch.empty((N, K), dtype=torch.uint8, device=x.device)
+    if sb is None:
+        sb = torch.empty(((N + 127) // 128, max(1, K // 128)), dtype=torch.float32, device=x.device)
+    _dev(q, torch.uint8, "q"), _dev(sb, torch.float32, "sb")
+    dev = _one_device(x=x, q=q, sb=sb)
+    with torch.cuda.device(dev):
+        _check(lib.fp8g_quantize_128x128(_ptr(x), _IN_DTYPE[x.dtype], N, K, _ptr(q), _ptr(sb),
+                                         _stream(stream, dev)), "fp8g_quantize_128x128")
+    return q, sb

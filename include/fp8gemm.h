@@ -175,6 +175,48 @@ int fp8_gemm_nt_no_alloc(const uint8_t *A, const float *sa, int ld_sa,
  */
 int fp8g_sa_to_mn_major(const float *src, float *dst, int G, int rows, int KB, int ld_sa);
 
+/*
+ * FP8 quantisers: the step before the GEMM that the pages leave to the caller
+ * (kakushin.no, "Hvorfor FP8 og FP4 er interessant": inputs must be converted
+ * to FP8 by the user), at the GEMM's granularity (GeekNews, "DeepSeek,
+ * DeepGEMM 오픈소스 공개", topic body, first bullet: fine-grained scaling).
+ * For every group G of input values:
+ *     scale = amax(|G|) / 448   in FP32 (448 = the largest finite e4m3 value;
+ *                               scale = 1 when every value of G is zero)
+ *     code  = e4m3 of the FP32 quotient x / scale, rounded to nearest even,
+ *             saturating at +-448 (one IEEE FP32 division per element).
+ * The outputs are the GEMM calls' inputs, in their layouts.  Inputs must be
+ * finite.  x_dtype is FP8G_IN_BF16 (x holds bf16 bit patterns) or
+ * FP8G_IN_F32.  All pointers are DEVICE pointers owned by the caller; x must
+ * not overlap the outputs.  The call enqueues one kernel on `stream` and
+ * returns without waiting; it reads no device memory on the host and
+ * allocates nothing.  Errors: FP8G_ERR_INVALID_ARG (null pointer, bad size
+ * or dtype), FP8G_ERR_MISALIGNED (x and q not 16-byte aligned, sa not
+ * 16-byte or sb not 4-byte aligned, ld_sa % 4 != 0), FP8G_ERR_CUDA (launch
+ * failed).  rows == 0 or N == 0 is a no-op.
+ */
+#define FP8G_IN_BF16 0
+#define FP8G_IN_F32 1
+
+/*
+ * Activations, one scale per 1x128 group of a row:
+ *   x [rows][K] (K % 128 == 0)  ->  q [rows][K] e4m3 codes,
+ *   sa [K/128][ld_sa] float, sa[kb*ld_sa + r] = scale of x[r, 128kb..+127]
+ *   (ld_sa >= rows, ld_sa % 4 == 0; entries past `rows` are not written).
+ */
+int fp8g_quantize_1x128(const void *x, int x_dtype, int rows, int K,
+                        uint8_t *q, float *sa, int ld_sa, cudaStream_t stream);
+
+/*
+ * Weights, one scale per 128x128 block:
+ *   x [N][K] (K % 128 == 0)  ->  q [N][K] e4m3 codes,
+ *   sb [ceil(N/128)][K/128] float, sb[nb*KB + kb] = scale of the block of
+ *   rows 128nb.. (fewer in the last block row when N % 128 != 0) and
+ *   columns 128kb..+127.
+ */
+int fp8g_quantize_128x128(const void *x, int x_dtype, int N, int K,
+                          uint8_t *q, float *sb, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *fp8g_status_string(int status);
 

@@ -26,14 +26,17 @@ def lib():
     return L
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def declared_functions(path=None):
+    """Functions declared by one header, or by every header under include/."""
+    import glob
+    paths = [path] if path else sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
+    text = "".join(open(p).read() for p in paths)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
 
 
 def test_header_declares_the_three_entry_points():
-    names = declared_functions()
+    names = declared_functions(HEADER)
     for n in ("fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked"):
         assert n in names
 
@@ -153,3 +156,12 @@ def test_sa_to_mn_major_round_trips_ragged_rows(lib):
     assert f(ptr(src), ptr(out), 1, 8, 3, 4) == 1       # ld_sa < rows
     assert f(ptr(src), ptr(out), 1, 4, 0, 4) == 1       # KB < 1
     assert f(ptr(src), ptr(out), 1, 5, 3, 6) == 2       # ld_sa % 4 != 0
+
+
+def test_testing_hook_argument_checks(lib):
+    f = lib.fp8g_testing_withhold_stage
+    f.argtypes = [C.c_int, C.c_uint]
+    assert f(3, 50) == 1            # limit below 100 us
+    assert f(3, 2_000_000) == 1     # limit above 1 s
+    assert f(3, 2000) == 0
+    assert f(-1, 0) == 0            # off again
