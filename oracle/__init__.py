@@ -39,6 +39,12 @@ def load(path: str):
     L.fp8o_quantize_1x128.argtypes = [P, i, i, P, P, i]
     L.fp8o_quantize_128x128.restype = i
     L.fp8o_quantize_128x128.argtypes = [P, i, i, P, P]
+    L.fp8o_moe_layout.restype = i
+    L.fp8o_moe_layout.argtypes = [P, i, i, i, P, P, P, P]
+    L.fp8o_moe_dispatch.restype = i
+    L.fp8o_moe_dispatch.argtypes = [P, i, i, P, i, i, i, P, P, i, P, P]
+    L.fp8o_moe_combine.restype = i
+    L.fp8o_moe_combine.argtypes = [P, i, P, P, i, i, P]
     return L
 
 
@@ -156,3 +162,46 @@ def quantize_128x128(x):
     if lib().fp8o_quantize_128x128(_p(x), int(N), int(K), _p(q), _p(sb)):
         raise ValueError("oracle: bad arguments")
     return q, sb
+
+
+def moe_layout(e, G, blocks):
+    """Expert layout of routed rows e [R] (int32; -1 = dropped).  Returns
+    (blocks_used, cnt [G], off [G], pos [R], m_indices [blocks])."""
+    e = _c(e, np.int32)
+    R = len(e)
+    cnt, off = np.zeros(G, np.int32), np.zeros(G, np.int32)
+    pos, mi = np.zeros(R, np.int32), np.zeros(blocks, np.int32)
+    used = lib().fp8o_moe_layout(_p(e), R, int(G), int(blocks), _p(cnt), _p(off), _p(pos), _p(mi))
+    if used < 0:
+        raise ValueError("oracle: bad arguments or too few blocks")
+    return used, cnt, off, pos, mi
+
+
+def moe_dispatch(x, e, topk, G, blocks, ld_sa=None, fill=0):
+    """Dispatch with quantisation: x [T, K] float32 token activations, e [T*topk].
+    Returns (blocks_used, A [blocks*128, K] uint8, sa [KB, ld_sa], pos, m_indices);
+    rows of unused blocks keep `fill`."""
+    x = _c(x, np.float32)
+    e = _c(e, np.int32)
+    T, K = x.shape
+    M = blocks * 128
+    ld = M if ld_sa is None else int(ld_sa)
+    A = np.full((M, K), fill, np.uint8)
+    sa = np.zeros((K // 128, ld), np.float32)
+    pos, mi = np.zeros(len(e), np.int32), np.zeros(blocks, np.int32)
+    used = lib().fp8o_moe_dispatch(_p(x), int(T), int(K), _p(e), int(topk), int(G), int(blocks),
+                                   _p(A), _p(sa), int(ld), _p(pos), _p(mi))
+    if used < 0:
+        raise ValueError("oracle: bad arguments or too few blocks")
+    return used, A, sa, pos, mi
+
+
+def moe_combine(D_bits, pos, w, T, topk):
+    """out [T, N] bf16 bits = bf16(sum_k w * D[pos]) in FP32, fused multiply-adds in slot order."""
+    D_bits = _c(D_bits, np.uint16)
+    pos = _c(pos, np.int32)
+    N = D_bits.shape[1]
+    wp = None if w is None else _c(w, np.float32)
+    out = np.zeros((T, N), np.uint16)
+    lib().fp8o_moe_combine(_p(D_bits), int(N), _p(pos), None if wp is None else _p(wp), int(T), int(topk), _p(out))
+    return out

@@ -399,3 +399,125 @@ int fp8o_quantize_128x128(const float *x, int N, int K, uint8_t *q, float *sb)
     }
     return 0;
 }
+
+/* ===========================================================================
+ * The expert pipeline on either side of the contiguous grouped GEMM (GeekNews
+ * page, "MoE 모델을 위한 그룹화 GEMM 성능": the contiguous layout groups the
+ * rows of A along M by expert, with N and K shared, one expert per 128-row
+ * block).  The pages describe only the layout; the steps below are its
+ * plainest construction (readings, since the pages give no algorithm):
+ *
+ *  dispatch: routed row r (r = t * topk + k: token t, slot k) goes to expert
+ *    e[r].  Expert g's rows, in increasing r, fill a segment padded to a
+ *    multiple of 128 rows; the segments follow each other in expert order
+ *    (off[g] = sum over g' < g of the padded counts).  Row r lands at
+ *    pos[r] = off[e[r]] + (number of r' < r with e[r'] == e[r]).  Block b of
+ *    the padded layout has m_indices[b] = its expert, or -1 past the last
+ *    segment (up to `blocks` entries).  Row pos[r] of A holds token t's
+ *    activations quantised per 1x128 group (the quantiser above); padding
+ *    rows hold zero codes and zero scales.
+ *  combine: out[t, n] = bf16_rne(acc), acc = sum over k of w[t*topk + k] *
+ *    D[pos[t*topk + k], n], accumulated in FP32 in slot order with one fused
+ *    multiply-add per slot (acc = fmaf(w, d, acc), acc starting at 0); D is
+ *    bf16.  w == NULL means every weight is 1.
+ * ======================================================================== */
+
+/* Layout only.  e [R] experts (0 <= e < G, -1 = row dropped: it gets
+ * pos = -1 and no place); outputs cnt [G], off [G], pos [R], m_indices
+ * [blocks].  Returns the number of 128-row blocks used, or -1 if they do not
+ * fit in `blocks` or an argument is bad. */
+int fp8o_moe_layout(const int32_t *e, int R, int G, int blocks,
+                    int32_t *cnt, int32_t *off, int32_t *pos, int32_t *m_indices)
+{
+    if (R < 0 || G < 1 || blocks < 0)
+        return -1;
+    for (int g = 0; g < G; ++g)
+        cnt[g] = 0;
+    for (int r = 0; r < R; ++r) {
+        if (e[r] >= G)
+            return -1;
+        if (e[r] >= 0)
+            cnt[e[r]]++;
+    }
+    long used = 0;
+    for (int g = 0; g < G; ++g) {
+        off[g] = (int32_t)(used * 128);
+        used += (cnt[g] + 127) / 128;
+    }
+    if (used > blocks)
+        return -1;
+    for (int b = 0; b < blocks; ++b)
+        m_indices[b] = -1;
+    for (int g = 0; g < G; ++g)
+        for (int b = off[g] / 128; b < off[g] / 128 + (cnt[g] + 127) / 128; ++b)
+            m_indices[b] = g;
+    int32_t *seen = (int32_t *)calloc((size_t)G, sizeof(int32_t));
+    for (int r = 0; r < R; ++r) {
+        if (e[r] < 0) {
+            pos[r] = -1;
+            continue;
+        }
+        pos[r] = off[e[r]] + seen[e[r]]++;
+    }
+    free(seen);
+    return (int)used;
+}
+
+/* Dispatch with quantisation: x [T][K] float (token activations), e [R]
+ * with R = T * topk.  Writes A [blocks*128][K] codes, sa [KB][ld_sa]
+ * (ld_sa >= blocks*128), pos [R], m_indices [blocks].  Rows of A in unused
+ * blocks are left as they are.  Returns the number of blocks used, or -1. */
+int fp8o_moe_dispatch(const float *x, int T, int K, const int32_t *e, int topk, int G, int blocks,
+                      uint8_t *A, float *sa, int ld_sa, int32_t *pos, int32_t *m_indices)
+{
+    if (T < 0 || topk < 1 || K <= 0 || K % 128 || ld_sa < blocks * 128)
+        return -1;
+    int R = T * topk, KB = K / 128;
+    int32_t *cnt = (int32_t *)malloc(sizeof(int32_t) * (size_t)G);
+    int32_t *off = (int32_t *)malloc(sizeof(int32_t) * (size_t)G);
+    int used = fp8o_moe_layout(e, R, G, blocks, cnt, off, pos, m_indices);
+    if (used >= 0) {
+        /* padding rows: zero codes, zero scales */
+        for (int g = 0; g < G; ++g)
+            for (long row = off[g] + cnt[g]; row < off[g] + (long)(cnt[g] + 127) / 128 * 128; ++row) {
+                memset(A + row * K, 0, (size_t)K);
+                for (int kb = 0; kb < KB; ++kb)
+                    sa[(long)kb * ld_sa + row] = 0.0f;
+            }
+        /* routed rows: the token's row quantised per 1x128 group */
+        float *rowsa = (float *)malloc(sizeof(float) * (size_t)KB);
+        for (int r = 0; r < R; ++r) {
+            if (pos[r] < 0)
+                continue;
+            fp8o_quantize_1x128(x + (long)(r / topk) * K, 1, K, A + (long)pos[r] * K, rowsa, 1);
+            for (int kb = 0; kb < KB; ++kb)
+                sa[(long)kb * ld_sa + pos[r]] = rowsa[kb];
+        }
+        free(rowsa);
+    }
+    free(cnt);
+    free(off);
+    return used;
+}
+
+/* Combine: D [rows][N] bf16 patterns, pos [T*topk], w [T*topk] or NULL ->
+ * out [T][N] bf16 patterns.  Slots with pos < 0 are skipped.  Returns 0. */
+int fp8o_moe_combine(const uint16_t *D, int N, const int32_t *pos, const float *w,
+                     int T, int topk, uint16_t *out)
+{
+    for (long t = 0; t < T; ++t)
+        for (int n = 0; n < N; ++n) {
+            float acc = 0.0f;
+            for (int k = 0; k < topk; ++k) {
+                long r = t * topk + k;
+                if (pos[r] < 0)
+                    continue;
+                uint32_t bits = (uint32_t)D[(long)pos[r] * N + n] << 16;
+                float d;
+                memcpy(&d, &bits, sizeof d);
+                acc = fmaf(w ? w[r] : 1.0f, d, acc);
+            }
+            out[t * N + n] = fp8o_bf16_rne((double)acc);
+        }
+    return 0;
+}

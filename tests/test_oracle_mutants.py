@@ -14,6 +14,7 @@ import oracle
 from oracle.build import SRC as ORACLE_SRC
 
 from . import test_oracle_pins as pins
+from . import test_oracle_moe_pins as mpins
 from . import test_oracle_quant_pins as qpins
 
 MUTANTS = {
@@ -43,6 +44,14 @@ MUTANTS = {
     "quant_sa_layout": ("sa[(long)kb * ld_sa + r] = s;", "sa[r * KB + kb] = s;"),
     "quant_block_rows": ("for (long r = r0; r < r1; ++r)\n                for (int j = 0; j < 128; ++j) {\n                    float v",
                          "for (long r = r0; r < r0 + 1; ++r)\n                for (int j = 0; j < 128; ++j) {\n                    float v"),
+    # the expert pipeline around the contiguous GEMM
+    "moe_unstable": ("pos[r] = off[e[r]] + seen[e[r]]++;", "pos[r] = off[e[r]] + (cnt[e[r]] - 1 - seen[e[r]]++);"),
+    "moe_extra_block": ("used += (cnt[g] + 127) / 128;", "used += (cnt[g] + 255) / 128;"),
+    "moe_m_indices_short": ("b < off[g] / 128 + (cnt[g] + 127) / 128; ++b)", "b < off[g] / 128 + cnt[g] / 128; ++b)"),
+    "moe_padding_half_zeroed": ("memset(A + row * K, 0, (size_t)K);", "memset(A + row * K, 0, (size_t)K / 2);"),
+    "moe_wrong_token": ("x + (long)(r / topk) * K", "x + (long)(r % topk) * K"),
+    "combine_no_weight": ("acc = fmaf(w ? w[r] : 1.0f, d, acc);", "acc = fmaf(1.0f, d, acc);"),
+    "combine_unfused": ("acc = fmaf(w ? w[r] : 1.0f, d, acc);", "acc = (w ? w[r] : 1.0f) * d + acc;"),
 }
 
 # every pin that takes no parameters, plus the parametrised ones at one or two points
@@ -70,6 +79,12 @@ PINS = [
     qpins.test_quantize_1x128_error_bound_and_locality,
     lambda: qpins.test_quantize_128x128_against_torch(200, 384),
     qpins.test_quantize_128x128_block_is_shared_by_its_rows_only,
+    lambda: mpins.test_layout_matches_a_stable_sort(300, 2, 5, 0.0),
+    lambda: mpins.test_layout_matches_a_stable_sort(1000, 8, 64, 0.1),
+    mpins.test_layout_rejects_too_few_blocks,
+    mpins.test_dispatch_rows_are_the_quantised_tokens_and_padding_is_zero,
+    mpins.test_combine_is_a_gather_for_one_slot_and_a_weighted_fma_chain,
+    mpins.test_combine_rounds_once_per_slot,
 ]
 
 
