@@ -476,6 +476,27 @@ int run(const Problem& P, cudaStream_t stream) {
 
 }  // namespace
 
+namespace fp8g {
+// Device address of this library's error word on the current device (looked
+// up once per device), for kernels of other translation units.
+uint32_t* device_error_word() {
+  static std::mutex mu;
+  static uint32_t* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fp8g_error_word) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = static_cast<uint32_t*>(p);
+  }
+  return addr[dev];
+}
+}  // namespace fp8g
+
 extern "C" {
 
 int fp8_gemm_nt(const uint8_t* A, const float* sa, int ld_sa, const uint8_t* B, const float* sb, uint16_t* D,

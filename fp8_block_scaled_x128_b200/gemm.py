@@ -38,6 +38,12 @@ lib.fp8g_quantize_128x128.restype = _I
 lib.fp8g_quantize_128x128.argtypes = [_P, _I, _I, _I, _P, _P, _P]
 lib.fp8g_testing_withhold_stage.restype = _I
 lib.fp8g_testing_withhold_stage.argtypes = [_I, C.c_uint]
+lib.fp8g_moe_dispatch_workspace_bytes.restype = C.c_size_t
+lib.fp8g_moe_dispatch_workspace_bytes.argtypes = [_I, _I]
+lib.fp8g_moe_dispatch.restype = _I
+lib.fp8g_moe_dispatch.argtypes = [_P, _I, _I, _I, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P, C.c_size_t, _P]
+lib.fp8g_moe_combine.restype = _I
+lib.fp8g_moe_combine.argtypes = [_P, _I, _P, _P, _I, _I, _P, _P]
 lib.fp8g_status_string.restype = C.c_char_p
 lib.fp8g_status_string.argtypes = [_I]
 lib.fp8g_get_device_error.restype = _I
@@ -53,7 +59,7 @@ lib.fp8g_last_variant.argtypes = []
 lib.fp8g_version.restype = _I
 lib.fp8g_version.argtypes = []
 
-DEVERR_TIMEOUT, DEVERR_BAD_M_INDEX, DEVERR_MASKED_OVER = 0x1, 0x2, 0x4
+DEVERR_TIMEOUT, DEVERR_BAD_M_INDEX, DEVERR_MASKED_OVER, DEVERR_BAD_EXPERT = 0x1, 0x2, 0x4, 0x8
 
 
 class Fp8GemmError(RuntimeError):
@@ -261,3 +267,59 @@ def quantize_128x128(x, q=None, sb=None, stream=None):
         _check(lib.fp8g_quantize_128x128(_ptr(x), _IN_DTYPE[x.dtype], N, K, _ptr(q), _ptr(sb),
                                          _stream(stream, dev)), "fp8g_quantize_128x128")
     return q, sb
+
+
+def moe_blocks(T: int, topk: int, G: int) -> int:
+    """128-row blocks of A that fit any routing of T*topk rows to G experts."""
+    return (T * topk + 127) // 128 + G
+
+
+def moe_dispatch(x, expert, topk, G, blocks=None, out=None, stream=None):
+    """Expert dispatch before the contiguous GEMM: x [T, K] (bfloat16 or float32),
+    expert [T*topk] int32 (-1 = dropped) -> (A [blocks*128, K] uint8, sa [K/128,
+    blocks*128] float32, pos [T*topk] int32, m_indices [blocks] int32).  `out`
+    may pass those four tensors (and a workspace as a fifth) to reuse them."""
+    _quant_input(x)
+    T, K = x.shape
+    R = T * topk
+    _dev(expert, torch.int32, "expert")
+    if expert.numel() != R:
+        raise ValueError(f"expert: {expert.numel()} entries for {T} tokens x topk {topk}")
+    nb = moe_blocks(T, topk, G) if blocks is None else int(blocks)
+    ws_bytes = lib.fp8g_moe_dispatch_workspace_bytes(R, G)
+    if ws_bytes == 0:
+        raise ValueError(f"moe_dispatch: unsupported R={R}, G={G} (1 <= G <= 256)")
+    if out is None:
+        A = torch.empty((nb * 128, K), dtype=torch.uint8, device=x.device)
+        sa = torch.empty((K // 128, nb * 128), dtype=torch.float32, device=x.device)
+        pos = torch.empty(max(R, 1), dtype=torch.int32, device=x.device)
+        mi = torch.empty(nb, dtype=torch.int32, device=x.device)
+        ws = torch.empty((ws_bytes + 3) // 4, dtype=torch.int32, device=x.device)
+    else:
+        A, sa, pos, mi, ws = out
+    dev = _one_device(x=x, expert=expert, A=A, sa=sa, pos=pos, m_indices=mi, workspace=ws)
+    with torch.cuda.device(dev):
+        _check(lib.fp8g_moe_dispatch(_ptr(x), _IN_DTYPE[x.dtype], T, K, _ptr(expert), int(topk), int(G), nb,
+                                     _ptr(A), _ptr(sa), sa.shape[-1], _ptr(pos), _ptr(mi), _ptr(ws),
+                                     ws.numel() * 4, _stream(stream, dev)), "fp8g_moe_dispatch")
+    return A, sa, pos[:R], mi
+
+
+def moe_combine(D, pos, w, T, topk, out=None, stream=None):
+    """Combine after the GEMM: out [T, N] bfloat16 = sum over slots of w * D[pos]
+    (FP32, one fused multiply-add per slot in slot order); w may be None."""
+    _dev(D, torch.bfloat16, "D"), _dev(pos, torch.int32, "pos")
+    N = D.shape[-1]
+    if w is not None:
+        _dev(w, torch.float32, "w")
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=D.device)
+    _dev(out, torch.bfloat16, "out")
+    tensors = dict(D=D, pos=pos, out=out)
+    if w is not None:
+        tensors["w"] = w
+    dev = _one_device(**tensors)
+    with torch.cuda.device(dev):
+        _check(lib.fp8g_moe_combine(_ptr(D), N, _ptr(pos), _ptr(w), int(T), int(topk), _ptr(out),
+                                    _stream(stream, dev)), "fp8g_moe_combine")
+    return out

@@ -53,6 +53,7 @@
 #ifndef FP8GEMM_H
 #define FP8GEMM_H
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -73,6 +74,7 @@ enum fp8g_status {
 #define FP8G_DEVERR_TIMEOUT       0x1u  /* a pipeline wait gave up; outputs of that call are invalid */
 #define FP8G_DEVERR_BAD_M_INDEX   0x2u  /* contiguous: m_indices entry >= G (block skipped) */
 #define FP8G_DEVERR_MASKED_OVER   0x4u  /* masked: masked_m[g] > Mmax (clamped to Mmax) */
+#define FP8G_DEVERR_BAD_EXPERT    0x8u  /* MoE dispatch: an expert id >= G or < -1 (row dropped) */
 
 /*
  * Dense NT GEMM (GeekNews page, "일반 GEMM 성능 (Dense 모델)").
@@ -216,6 +218,65 @@ int fp8g_quantize_1x128(const void *x, int x_dtype, int rows, int K,
  */
 int fp8g_quantize_128x128(const void *x, int x_dtype, int N, int K,
                           uint8_t *q, float *sb, cudaStream_t stream);
+
+/*
+ * The expert pipeline around the contiguous grouped GEMM.  The pages describe
+ * only the layout the GEMM consumes (GeekNews, "MoE 모델을 위한 그룹화 GEMM
+ * 성능": rows of A grouped along M by expert, N and K shared, each expert's
+ * segment a whole number of 128-row blocks); these two calls build it from a
+ * router's output and bring the GEMM's rows back to their tokens:
+ *
+ *   x [T][K] token activations --fp8g_moe_dispatch--> A, sa, m_indices, pos
+ *   --m_grouped_fp8_gemm_nt_contiguous(M = blocks*128)--> D [blocks*128][N]
+ *   --fp8g_moe_combine--> out [T][N]
+ *
+ * Routed row r = t*topk + k is slot k of token t; expert[r] is its expert in
+ * [0, G), or -1 if it is dropped.  Expert g's rows keep their order r and fill
+ * a segment padded up to a multiple of 128 rows; the segments follow each
+ * other in expert order from row 0; pos[r] is row r's row in A (-1 if
+ * dropped).  m_indices[b] is the expert of block b, -1 for the unused blocks
+ * after the last segment (the GEMM skips them).  Nothing is read back on the
+ * host, so with a fixed `blocks` the three calls can be captured in one CUDA
+ * graph.  All pointers are DEVICE pointers owned by the caller; the calls
+ * enqueue kernels on `stream` and return without waiting.
+ */
+
+/* Bytes of workspace fp8g_moe_dispatch needs for R = T*topk routed rows and
+ * G experts (4 * (ceil(R/1024)*G + 2G)); 0 for bad arguments. */
+size_t fp8g_moe_dispatch_workspace_bytes(int R, int G);
+
+/*
+ * Dispatch: builds the contiguous layout and quantises each routed row's
+ * token into it, per 1x128 group (as fp8g_quantize_1x128).
+ *   x [T][K] (bf16 patterns or FP32, x_dtype), K % 128 == 0, K <= 65536;
+ *   expert [T*topk] int32; topk >= 1; 1 <= G <= 256;
+ *   blocks >= ceil(T*topk/128) + G (room for any routing);
+ *   outputs A [blocks*128][K] e4m3 codes, sa [K/128][ld_sa] (ld_sa >=
+ *   blocks*128, ld_sa % 4 == 0), pos [T*topk], m_indices [blocks];
+ *   workspace: >= fp8g_moe_dispatch_workspace_bytes(T*topk, G) bytes,
+ *   4-byte aligned, overwritten.
+ * Padding rows of every segment get zero codes and zero scales (their D rows
+ * are zero); rows of unused blocks are not written.  An expert id out of
+ * range drops the row and sets FP8G_DEVERR_BAD_EXPERT.
+ * Errors: FP8G_ERR_INVALID_ARG (bad size, capacity or workspace, null
+ * pointer), FP8G_ERR_MISALIGNED (x, A, sa not 16-byte aligned; ld_sa), and
+ * FP8G_ERR_CUDA.
+ */
+int fp8g_moe_dispatch(const void *x, int x_dtype, int T, int K,
+                      const int32_t *expert, int topk, int G, int blocks,
+                      uint8_t *A, float *sa, int ld_sa, int32_t *pos, int32_t *m_indices,
+                      void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Combine: out[t][n] = bf16_rne(acc), acc = sum over k of w[t*topk + k] *
+ * D[pos[t*topk + k]][n], accumulated in FP32 in slot order with one fused
+ * multiply-add per slot (acc starts at 0; slots with pos < 0 are skipped;
+ * w == NULL means weights of 1).  D [*][N] and out [T][N] are bf16 patterns,
+ * N % 8 == 0, both 16-byte aligned.  With topk == 1 and w == NULL it returns
+ * the GEMM's rows to token order.
+ */
+int fp8g_moe_combine(const uint16_t *D, int N, const int32_t *pos, const float *w,
+                     int T, int topk, uint16_t *out, cudaStream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char *fp8g_status_string(int status);
