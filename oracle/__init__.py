@@ -45,6 +45,8 @@ def load(path: str):
     L.fp8o_moe_dispatch.argtypes = [P, i, i, P, i, i, i, P, P, i, P, P]
     L.fp8o_moe_combine.restype = i
     L.fp8o_moe_combine.argtypes = [P, i, P, P, i, i, P]
+    L.fp8o_bf16_gemm_nt.restype = i
+    L.fp8o_bf16_gemm_nt.argtypes = [P, P, i, i, i, P, i, P, P]
     return L
 
 
@@ -205,3 +207,18 @@ def moe_combine(D_bits, pos, w, T, topk):
     out = np.zeros((T, N), np.uint16)
     lib().fp8o_moe_combine(_p(D_bits), int(N), _p(pos), None if wp is None else _p(wp), int(T), int(topk), _p(out))
     return out
+
+
+def bf16_gemm_nt(A_bits, B_bits, rows=None):
+    """BF16 NT GEMM: A [M, K], B [N, K] bf16 bit patterns (uint16).  Returns
+    (exact float64 [nrows, N], bf16 bits [nrows, N])."""
+    A, B = _c(A_bits, np.uint16), _c(B_bits, np.uint16)
+    M, K = A.shape
+    N = B.shape[0]
+    r = None if rows is None else _c(rows, np.int32)
+    nrows = M if r is None else len(r)
+    ex = np.zeros((nrows, N), np.float64)
+    bf = np.zeros((nrows, N), np.uint16)
+    if lib().fp8o_bf16_gemm_nt(_p(A), _p(B), int(M), int(N), int(K), _p(r), int(nrows), _p(ex), _p(bf)):
+        raise ValueError("oracle: bad arguments")
+    return ex, bf

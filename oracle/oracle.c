@@ -521,3 +521,50 @@ int fp8o_moe_combine(const uint16_t *D, int N, const int32_t *pos, const float *
         }
     return 0;
 }
+
+/* ===========================================================================
+ * BF16 NT GEMM, the other input format the pages list for the library
+ * (kakushin.no, "Hva gjør DeepGEMM?": FP8, FP4 and BF16 computations):
+ *   D[m,n] = bf16_rne( sum_k A[m,k] * B[n,k] ),  A [M][K], B [N][K] bf16.
+ * Each product of two bf16 values is exact in double (8 + 8 significant
+ * bits); the K-term sum is accumulated in double in k order (relative error
+ * far below the bf16 output's 2^-9) and rounded once to bf16.  Returns the
+ * unrounded sums and their bf16 patterns for the rows listed (NULL = all).
+ * ======================================================================== */
+static double bf16_value(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+int fp8o_bf16_gemm_nt(const uint16_t *A, const uint16_t *B, int M, int N, int K,
+                      const int *rows, int nrows, double *out_exact, uint16_t *out_bf16)
+{
+    if (M < 0 || N < 0 || K < 0)
+        return -1;
+    if (!rows)
+        nrows = M;
+    double *arow = (double *)malloc(sizeof(double) * (size_t)(K ? K : 1));
+    for (int i = 0; i < nrows; ++i) {
+        int m = rows ? rows[i] : i;
+        if (m < 0 || m >= M) {
+            free(arow);
+            return -1;
+        }
+        for (int k = 0; k < K; ++k)
+            arow[k] = bf16_value(A[(long)m * K + k]);
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k)
+                acc += arow[k] * bf16_value(B[(long)n * K + k]);
+            if (out_exact)
+                out_exact[(long)i * N + n] = acc;
+            if (out_bf16)
+                out_bf16[(long)i * N + n] = fp8o_bf16_rne(acc);
+        }
+    }
+    free(arow);
+    return 0;
+}

@@ -14,6 +14,7 @@ import oracle
 from oracle.build import SRC as ORACLE_SRC
 
 from . import test_oracle_pins as pins
+from . import test_oracle_bf16_pins as bpins
 from . import test_oracle_moe_pins as mpins
 from . import test_oracle_quant_pins as qpins
 
@@ -52,6 +53,9 @@ MUTANTS = {
     "moe_wrong_token": ("x + (long)(r / topk) * K", "x + (long)(r % topk) * K"),
     "combine_no_weight": ("acc = fmaf(w ? w[r] : 1.0f, d, acc);", "acc = fmaf(1.0f, d, acc);"),
     "combine_unfused": ("acc = fmaf(w ? w[r] : 1.0f, d, acc);", "acc = (w ? w[r] : 1.0f) * d + acc;"),
+    # the BF16 GEMM
+    "bf16_k_short": ("for (int k = 0; k < K; ++k)\n                acc += arow[k]", "for (int k = 0; k < K - 1; ++k)\n                acc += arow[k]"),
+    "bf16_b_transposed": ("bf16_value(B[(long)n * K + k])", "bf16_value(B[(long)k * N + n])"),
 }
 
 # every pin that takes no parameters, plus the parametrised ones at one or two points
@@ -85,6 +89,9 @@ PINS = [
     mpins.test_dispatch_rows_are_the_quantised_tokens_and_padding_is_zero,
     mpins.test_combine_is_a_gather_for_one_slot_and_a_weighted_fma_chain,
     mpins.test_combine_rounds_once_per_slot,
+    lambda: bpins.test_bf16_gemm_matches_numpy(33, 40, 256),
+    bpins.test_bf16_gemm_exact_integers,
+    bpins.test_bf16_gemm_closed_forms,
 ]
 
 
