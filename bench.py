@@ -476,6 +476,90 @@ def e2e_measure(S: Shape, steps: int, stream, world: int) -> dict:
             "note": "pinned host inputs copied to the device, GEMM through the C ABI, D copied back, every step"}
 
 
+def measure_extras(dev, stream, sampler, steps: int) -> dict:
+    """The pieces around the GEMM, each timed in the same run on seeded
+    synthetic inputs larger than L2: the FP8 quantisers, the expert dispatch and
+    combine of the contiguous layout (a routing of 8192 tokens x top-4 over 4
+    experts, the contiguous workload's 32768 rows) and the BF16 GEMM.  Each
+    entry: device time per call (CUDA events over `steps` back-to-back calls
+    after warm-up) and its roofline against the measured peaks."""
+    import torch
+    from fp8_block_scaled_x128_b200 import gemm
+    pk = peaks()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    out = {}
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize(dev)
+            t0 = time.time()
+            while time.time() - t0 < 0.3:
+                fn()
+                torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0 = time.time()
+            e0.record(stream)
+            for _ in range(steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / steps * 1e-3, sampler.summary(s0 - 0.3, time.time())
+
+    def hbm(name, nbytes, fn, what):
+        sec, clk = timed(fn)
+        gbs = nbytes / sec / 1e9
+        out[name] = {"what": what, "us_per_call": sec * 1e6, "roofline": {
+            "bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
+            "algorithmic_bytes_per_call": nbytes, "peak_source": f"hbm_gbs of {pk['source']}"}, "clocks": clk}
+
+    # quantisers: bf16 activations [32768, 7168] and 4 experts' weights [16384, 7168]
+    T, K, N, G, topk = 8192, 7168, 4096, 4, 4
+    x = torch.randn(4 * T, K, generator=gen, device=dev).to(torch.bfloat16)
+    q, sa = gemm.quantize_1x128(x)
+    hbm("quantize_1x128_bf16_32768x7168", x.numel() * 3 + sa.numel() * 4,
+        lambda: gemm.quantize_1x128(x, q, sa, stream=stream), "activations, one scale per 1x128 group")
+    w = (torch.randn(G * N, K, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+    qb, sb = gemm.quantize_128x128(w)
+    hbm("quantize_128x128_bf16_16384x7168", w.numel() * 3 + sb.numel() * 4,
+        lambda: gemm.quantize_128x128(w, qb, sb, stream=stream), "weights, one scale per 128x128 block")
+    del x, q, sa, w, qb, sb
+    # expert dispatch + combine around the contiguous GEMM
+    xt = torch.randn(T, K, generator=gen, device=dev).to(torch.bfloat16)
+    e = torch.stack([torch.randperm(G, generator=gen, device=dev) for _ in range(T)]).to(torch.int32).reshape(-1)
+    R = T * topk
+    bufs = list(gemm.moe_dispatch(xt, e, topk, G))
+    ws = torch.empty((gemm.lib.fp8g_moe_dispatch_workspace_bytes(R, G) + 3) // 4, dtype=torch.int32, device=dev)
+    outs = (bufs[0], bufs[1], torch.empty(R, dtype=torch.int32, device=dev), bufs[3], ws)
+    hbm("moe_dispatch_8192x4_g4_k7168", T * K * 2 + R * K + R * (K // 128) * 4 + 2 * R * 4,
+        lambda: gemm.moe_dispatch(xt, e, topk, G, out=outs, stream=stream),
+        "routing -> contiguous layout, tokens quantised into it (counts, ranks, gather, padding)")
+    pos = outs[2]
+    Dm = torch.randn(bufs[0].shape[0], N, generator=gen, device=dev).to(torch.bfloat16)
+    wts = torch.rand(R, generator=gen, device=dev)
+    comb = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+    hbm("moe_combine_8192x4_n4096", R * N * 2 + T * N * 2 + R * 8,
+        lambda: gemm.moe_combine(Dm, pos, wts, T, topk, out=comb, stream=stream),
+        "GEMM rows back to tokens, weighted FP32 sum over the top-4 slots")
+    del xt, e, bufs, outs, Dm, wts, comb
+    # BF16 GEMM 8192^3 against the measured bf16 peak
+    Mb = 8192
+    A = torch.randn(Mb, Mb, generator=gen, device=dev).to(torch.bfloat16)
+    B = (torch.randn(Mb, Mb, generator=gen, device=dev) * 0.05).to(torch.bfloat16)
+    Db = torch.empty(Mb, Mb, dtype=torch.bfloat16, device=dev)
+    sec, clk = timed(lambda: gemm.bf16_gemm_nt(A, B, Db, stream=stream))
+    tf = 2.0 * Mb ** 3 / sec / 1e12
+    out["bf16_gemm_8192x8192x8192"] = {"what": "BF16 NT GEMM, FP32 accumulation", "us_per_call": sec * 1e6,
+                                       "variant": gemm.variant_names()[gemm.last_variant()], "roofline": {
+        "bound": "tensor", "achieved": tf, "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tf / pk["bf16"],
+        "peak_source": f"bf16_tflops (burst) of {pk['source']}"}, "clocks": clk}
+    del A, B, Db
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank: int, world: int) -> None:
     import torch
 
@@ -529,6 +613,7 @@ def run_ours(args, rank: int, world: int) -> None:
                     "gpu_launches": world * ps_steps * kernels_per_call(ps_variant),
                     "clocks": ps_clocks, "cpu_baseline": ps_cpu,
                 }
+        extras = {} if args.no_extras else measure_extras(dev, stream, sampler, max(args.steps, 10))
     finally:
         sampler.stop()
 
@@ -553,6 +638,8 @@ def run_ours(args, rank: int, world: int) -> None:
         line["cpu_baseline"] = headline_cpu
     if per_shape:
         line["per_shape"] = per_shape
+    if extras:
+        line["extras"] = extras
     print(json.dumps(line), flush=True)
 
 
@@ -567,6 +654,7 @@ def main() -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-shape", action="store_true", help="measure the headline workload only")
+    ap.add_argument("--no-extras", action="store_true", help="skip the quantiser / MoE / BF16 measurements")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi clocks (diagnostic)")
     ap.add_argument("--per-launch-events", action="store_true",
                     help="record an event between launches (diagnostic; prevents launch overlap)")

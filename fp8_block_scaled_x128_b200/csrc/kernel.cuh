@@ -81,7 +81,7 @@
 
 namespace fp8g {
 
-enum Kind : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+enum Kind : int { kDense = 0, kContiguous = 1, kMasked = 2, kBf16Dense = 3 };
 
 constexpr int kThreads = 384;
 constexpr int kIssuersPerWarp = 4;                  // TMA-issuing lanes in each producer warp

@@ -44,6 +44,8 @@ lib.fp8g_moe_dispatch.restype = _I
 lib.fp8g_moe_dispatch.argtypes = [_P, _I, _I, _I, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P, C.c_size_t, _P]
 lib.fp8g_moe_combine.restype = _I
 lib.fp8g_moe_combine.argtypes = [_P, _I, _P, _P, _I, _I, _P, _P]
+lib.bf16_gemm_nt.restype = _I
+lib.bf16_gemm_nt.argtypes = [_P, _P, _P, _I, _I, _I, _P]
 lib.fp8g_status_string.restype = C.c_char_p
 lib.fp8g_status_string.argtypes = [_I]
 lib.fp8g_get_device_error.restype = _I
@@ -323,3 +325,17 @@ def moe_combine(D, pos, w, T, topk, out=None, stream=None):
         _check(lib.fp8g_moe_combine(_ptr(D), N, _ptr(pos), _ptr(w), int(T), int(topk), _ptr(out),
                                     _stream(stream, dev)), "fp8g_moe_combine")
     return out
+
+
+def bf16_gemm_nt(A, B, D=None, stream=None):
+    """BF16 NT GEMM: A [M, K], B [N, K] bfloat16 -> D [M, N] bfloat16 (FP32 accumulation)."""
+    _dev(A, torch.bfloat16, "A"), _dev(B, torch.bfloat16, "B")
+    M, K = A.shape
+    N = B.shape[0]
+    if D is None:
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _dev(D, torch.bfloat16, "D")
+    dev = _one_device(A=A, B=B, D=D)
+    with torch.cuda.device(dev):
+        _check(lib.bf16_gemm_nt(_ptr(A), _ptr(B), _ptr(D), M, N, K, _stream(stream, dev)), "bf16_gemm_nt")
+    return D

@@ -278,6 +278,19 @@ int fp8g_moe_dispatch(const void *x, int x_dtype, int T, int K,
 int fp8g_moe_combine(const uint16_t *D, int N, const int32_t *pos, const float *w,
                      int T, int topk, uint16_t *out, cudaStream_t stream);
 
+/*
+ * BF16 NT GEMM on the same pipeline, the other input format the pages list
+ * next to FP8 (kakushin.no, "Hva gjør DeepGEMM?"):
+ *   D[m,n] = bf16_rne( sum_k A[m,k] * B[n,k] )   with FP32 accumulation,
+ *   A [M,K], B [N,K], D [M,N] bf16 bit patterns, row-major and dense.
+ * Requirements: K > 0, K % 64 == 0, K <= 65536, M, N >= 0, N % 8 == 0;
+ * A, B, D 16-byte aligned (FP8G_ERR_INVALID_ARG / FP8G_ERR_MISALIGNED
+ * otherwise).  Same conventions as fp8_gemm_nt: device pointers owned by the
+ * caller, one kernel enqueued on `stream`, nothing read on the host.
+ */
+int bf16_gemm_nt(const uint16_t *A, const uint16_t *B, uint16_t *D,
+                 int M, int N, int K, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *fp8g_status_string(int status);
 

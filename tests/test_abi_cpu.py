@@ -123,8 +123,8 @@ def test_every_variant_name_starts_with_its_kind(lib):
     # call's kind; a variant outside the three prefixes would go untested
     names = [lib.fp8g_variant_name(i).decode() for i in range(lib.fp8g_num_variants())]
     for n in names:
-        assert n.split("_", 1)[0] in ("dense", "contiguous", "masked"), n
-    for kind in ("dense", "contiguous", "masked"):
+        assert n.split("_", 1)[0] in ("dense", "contiguous", "masked", "bf16"), n
+    for kind in ("dense", "contiguous", "masked", "bf16"):
         assert any(n.startswith(kind + "_") for n in names), kind
 
 
@@ -165,3 +165,13 @@ def test_testing_hook_argument_checks(lib):
     assert f(3, 2_000_000) == 1     # limit above 1 s
     assert f(3, 2000) == 0
     assert f(-1, 0) == 0            # off again
+
+
+def test_bf16_host_validation(lib):
+    f = lib.bf16_gemm_nt
+    f.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p]
+    assert f(A, B, D, 64, 256, 96, S) == 1          # K % 64 != 0
+    assert f(A, B, D, 64, 250, 128, S) == 2         # N % 8 != 0
+    assert f(A + 8, B, D, 64, 256, 128, S) == 2     # A not 16-byte aligned
+    assert f(None, B, D, 64, 256, 128, S) == 1      # null A
+    assert f(None, None, None, 0, 256, 128, S) == 0  # M == 0: no-op
