@@ -47,6 +47,10 @@ def load(path: str):
     L.fp8o_moe_combine.argtypes = [P, i, P, P, i, i, P]
     L.fp8o_bf16_gemm_nt.restype = i
     L.fp8o_bf16_gemm_nt.argtypes = [P, P, i, i, i, P, i, P, P]
+    L.fp8o_ue8m0_value.restype = C.c_double
+    L.fp8o_ue8m0_value.argtypes = [C.c_uint8]
+    L.fp8o_gemm_nt_ue8m0.restype = i
+    L.fp8o_gemm_nt_ue8m0.argtypes = [P, P, i, P, P, i, i, i, P, i, P, P, i]
     return L
 
 
@@ -220,5 +224,24 @@ def bf16_gemm_nt(A_bits, B_bits, rows=None):
     ex = np.zeros((nrows, N), np.float64)
     bf = np.zeros((nrows, N), np.uint16)
     if lib().fp8o_bf16_gemm_nt(_p(A), _p(B), int(M), int(N), int(K), _p(r), int(nrows), _p(ex), _p(bf)):
+        raise ValueError("oracle: bad arguments")
+    return ex, bf
+
+
+def ue8m0_value(e: int) -> float:
+    return lib().fp8o_ue8m0_value(int(e))
+
+
+def gemm_nt_ue8m0(A, sfa, ld_sf, B, sfb, M, N, K, rows=None, nthreads=None):
+    """Dense NT GEMM with power-of-two scale bytes (UE8M0: 2^(e-127)).
+    Returns (exact float64 [nrows, N], bf16 bits [nrows, N])."""
+    A, B = _c(A, np.uint8), _c(B, np.uint8)
+    sfa, sfb = _c(sfa, np.uint8), _c(sfb, np.uint8)
+    r = None if rows is None else _c(rows, np.int32)
+    nrows = M if r is None else len(r)
+    ex = np.zeros((nrows, N), np.float64)
+    bf = np.zeros((nrows, N), np.uint16)
+    if lib().fp8o_gemm_nt_ue8m0(_p(A), _p(sfa), int(ld_sf), _p(B), _p(sfb), int(M), int(N), int(K), _p(r),
+                                int(nrows), _p(ex), _p(bf), int(nthreads or default_threads())):
         raise ValueError("oracle: bad arguments")
     return ex, bf

@@ -568,3 +568,40 @@ int fp8o_bf16_gemm_nt(const uint16_t *A, const uint16_t *B, int M, int N, int K,
     free(arow);
     return 0;
 }
+
+/* ===========================================================================
+ * Power-of-two (UE8M0) scales: the scale format of the block-scaled FP8
+ * tensor-core instructions that the SM100 generation the pages list adds
+ * (kakushin.no, requirements list: SM90 and SM100; the power-of-two scale
+ * format is the OCP microscaling E8M0 one).  A scale byte e stands for
+ * 2^(e - 127); e = 255 is NaN.  Same granularity and definition as the FP32
+ * scales above:
+ *   D[m,n] = bf16_rne( sum_kb ( sum_{k in kb} A[m,k] B[n,k] )
+ *                             * 2^(ea[kb][m] - 127) * 2^(eb[n/128][kb] - 127) )
+ * sfa [KB][ld_sf] bytes (MN-major like sa), sfb [NB][KB] bytes.  The powers
+ * of two are exact in float, so the FP32-scale definition is evaluated on
+ * the decoded scales.
+ * ======================================================================== */
+double fp8o_ue8m0_value(uint8_t e)
+{
+    return e == 255 ? NAN : ldexp(1.0, (int)e - 127);
+}
+
+int fp8o_gemm_nt_ue8m0(const uint8_t *A, const uint8_t *sfa, int ld_sf, const uint8_t *B,
+                       const uint8_t *sfb, int M, int N, int K, const int *rows, int nrows,
+                       double *out_exact, uint16_t *out_bf16, int nthreads)
+{
+    if (K <= 0 || K % 128 || M < 0 || N < 0 || ld_sf < M)
+        return -1;
+    int KB = K / 128, NB = (N + 127) / 128;
+    float *sa = (float *)malloc(sizeof(float) * (size_t)KB * (size_t)(ld_sf ? ld_sf : 1));
+    float *sb = (float *)malloc(sizeof(float) * (size_t)NB * (size_t)KB + 1);
+    for (long i = 0; i < (long)KB * ld_sf; ++i)
+        sa[i] = (float)fp8o_ue8m0_value(sfa[i]);
+    for (long i = 0; i < (long)NB * KB; ++i)
+        sb[i] = (float)fp8o_ue8m0_value(sfb[i]);
+    int rc = fp8o_gemm_nt(A, sa, ld_sf, B, sb, M, N, K, rows, nrows, out_exact, out_bf16, nthreads);
+    free(sa);
+    free(sb);
+    return rc;
+}

@@ -17,6 +17,7 @@ from . import test_oracle_pins as pins
 from . import test_oracle_bf16_pins as bpins
 from . import test_oracle_moe_pins as mpins
 from . import test_oracle_quant_pins as qpins
+from . import test_oracle_ue8m0_pins as upins
 
 MUTANTS = {
     "decode_bias": ("v = ldexp(8.0 + (double)m, e - 7 - 3);", "v = ldexp(8.0 + (double)m, e - 8 - 3);"),
@@ -56,6 +57,9 @@ MUTANTS = {
     # the BF16 GEMM
     "bf16_k_short": ("for (int k = 0; k < K; ++k)\n                acc += arow[k]", "for (int k = 0; k < K - 1; ++k)\n                acc += arow[k]"),
     "bf16_b_transposed": ("bf16_value(B[(long)n * K + k])", "bf16_value(B[(long)k * N + n])"),
+    # power-of-two scales
+    "ue8m0_bias": ("return e == 255 ? NAN : ldexp(1.0, (int)e - 127);", "return e == 255 ? NAN : ldexp(1.0, (int)e - 126);"),
+    "ue8m0_sfb_unused": ("sb[i] = (float)fp8o_ue8m0_value(sfb[i]);", "sb[i] = 1.0f;"),
 }
 
 # every pin that takes no parameters, plus the parametrised ones at one or two points
@@ -92,6 +96,9 @@ PINS = [
     lambda: bpins.test_bf16_gemm_matches_numpy(33, 40, 256),
     bpins.test_bf16_gemm_exact_integers,
     bpins.test_bf16_gemm_closed_forms,
+    upins.test_ue8m0_decode,
+    upins.test_ue8m0_gemm_matches_bruteforce,
+    upins.test_ue8m0_gemm_exact,
 ]
 
 
