@@ -16,6 +16,7 @@
 #include "kernel.cuh"
 #include "kernel_pair.cuh"
 #include "kernel_bf16.cuh"
+#include "kernel_ue8m0.cuh"
 
 using namespace fp8g;
 
@@ -51,6 +52,12 @@ Variant make_bf16_variant(const char* name) {
                  Bf16Layout<STAGES, kTmaStore>::kSmemAlloc, true, kBf16Threads, 0};
 }
 
+template <int STAGES>
+Variant make_ue8m0_variant(const char* name) {
+  return Variant{name, kUe8m0Dense, false, 256, STAGES, 1, false, &fp8_gemm_ue8m0_kernel<STAGES>,
+                 Ue8Layout<STAGES>::kSmemAlloc, false, kUe8Threads, 0};
+}
+
 template <int KIND, int STAGES, int BN, int OPT = 0, int NWG = default_nwg(BN)>
 Variant make_pair_variant(const char* name) {
   using S = PairShape<BN, NWG>;
@@ -79,6 +86,7 @@ const Variant kVariants[] = {
     make_pair_variant<kMasked, 6, 192>("masked_mlanes_pair_bn192_st6"),
     make_bf16_variant<6, false>("bf16_pair_bn256_st6"),
     make_bf16_variant<6, true>("bf16_pair_bn256_st6_tmastore"),
+    make_ue8m0_variant<4>("ue8m0_mlanes_bn256_st4"),
 };
 constexpr int kNumVariants = static_cast<int>(sizeof(kVariants) / sizeof(kVariants[0]));
 enum : int {
@@ -98,6 +106,7 @@ enum : int {
   V_MASKED_PAIR192,
   V_BF16,
   V_BF16_TMASTORE,
+  V_UE8M0,
   V_COUNT
 };
 static_assert(V_COUNT == kNumVariants, "variant table and names");
@@ -536,6 +545,58 @@ int launch_bf16(const uint16_t* A, const uint16_t* B, uint16_t* D, int M, int N,
   return FP8G_OK;
 }
 
+// FP8 GEMM with UE8M0 scales: one CTA per 128 x 256 tile, block-scaled MMA.
+int launch_ue8m0(const uint8_t* A, const uint8_t* sfa, int ld_sf, const uint8_t* B, const uint8_t* sfb, uint16_t* D,
+                 int M, int N, int K, int v, DeviceInfo* dev, cudaStream_t stream) {
+  const Variant& V = kVariants[v];
+  if (V.kind != kUe8m0Dense) return FP8G_ERR_UNSUPPORTED;
+  int rc = prepare_variant(dev, v);
+  if (rc) return rc;
+  Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.KB = K / 128;
+  p.NB = (N + 127) / 128;
+  p.G = 1;
+  p.n_tiles = (N + 255) / 256;
+  p.m_tiles = (M + 127) / 128;
+  p.num_tiles = p.n_tiles * p.m_tiles;
+  p.D = D;
+  p.ld_sa = ld_sf;
+  p.sfa = sfa;
+  p.sfb = sfb;
+  p.wait_limit_us = kWaitLimitUs;
+  p.test_withhold_it = -1;
+  CUtensorMap tmA, tmB, tmD;
+  rc = encode3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, 1, (uint64_t)K, (uint64_t)K * M, 128, 128,
+                CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!rc)
+    rc = encode3d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, 1, (uint64_t)K, (uint64_t)K * N, 128, 256,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!rc)
+    rc = encode3d(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, N, M, 1, (uint64_t)N * 2, (uint64_t)N * 2 * M, 32, 32,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(std::min(p.num_tiles, dev->sms), 1, 1);
+  cfg.blockDim = dim3(V.threads, 1, 1);
+  cfg.dynamicSmemBytes = V.smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  void* args[] = {&tmA, &tmB, &tmD, &p};
+  if (cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(V.fn), args) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FP8G_ERR_CUDA;
+  }
+  t_last_variant = v;
+  return FP8G_OK;
+}
+
 int run(const Problem& P, cudaStream_t stream) {
   DeviceInfo* dev = nullptr;
   int rc = device_info(&dev);
@@ -634,6 +695,19 @@ int bf16_gemm_nt(const uint16_t* A, const uint16_t* B, uint16_t* D, int M, int N
   // 861 vs 871 us; 4096 x 7168 x 16384: 766 vs 791 us)
   const int v = ov >= 0 ? ov : V_BF16_TMASTORE;
   return launch_bf16(A, B, D, M, N, K, v, dev, stream);
+}
+
+int fp8_gemm_nt_ue8m0(const uint8_t* A, const uint8_t* sfa, int ld_sf, const uint8_t* B, const uint8_t* sfb,
+                      uint16_t* D, int M, int N, int K, cudaStream_t stream) {
+  int rc = check_shapes(M, N, K, ld_sf);
+  if (rc) return rc;
+  if (M == 0 || N == 0) return FP8G_OK;
+  if (!A || !sfa || !B || !sfb || !D) return FP8G_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16)) return FP8G_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev))) return rc;
+  const int ov = g_override.load(std::memory_order_relaxed);
+  return launch_ue8m0(A, sfa, ld_sf, B, sfb, D, M, N, K, ov >= 0 ? ov : V_UE8M0, dev, stream);
 }
 
 const char* fp8g_status_string(int status) {

@@ -81,7 +81,7 @@
 
 namespace fp8g {
 
-enum Kind : int { kDense = 0, kContiguous = 1, kMasked = 2, kBf16Dense = 3 };
+enum Kind : int { kDense = 0, kContiguous = 1, kMasked = 2, kBf16Dense = 3, kUe8m0Dense = 4 };
 
 constexpr int kThreads = 384;
 constexpr int kIssuersPerWarp = 4;                  // TMA-issuing lanes in each producer warp
@@ -118,6 +118,9 @@ struct Params {
   // runs out without any fault
   uint32_t wait_limit_us;
   int test_withhold_it;
+  // power-of-two scale bytes of the UE8M0 GEMM: sfa [KB][ld_sa], sfb [NB][KB]
+  const uint8_t* sfa;
+  const uint8_t* sfb;
 };
 
 // SPLIT template values selecting the global-memory split-K (count at run

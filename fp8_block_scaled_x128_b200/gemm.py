@@ -46,6 +46,8 @@ lib.fp8g_moe_combine.restype = _I
 lib.fp8g_moe_combine.argtypes = [_P, _I, _P, _P, _I, _I, _P, _P]
 lib.bf16_gemm_nt.restype = _I
 lib.bf16_gemm_nt.argtypes = [_P, _P, _P, _I, _I, _I, _P]
+lib.fp8_gemm_nt_ue8m0.restype = _I
+lib.fp8_gemm_nt_ue8m0.argtypes = [_P, _P, _I, _P, _P, _P, _I, _I, _I, _P]
 lib.fp8g_status_string.restype = C.c_char_p
 lib.fp8g_status_string.argtypes = [_I]
 lib.fp8g_get_device_error.restype = _I
@@ -338,4 +340,21 @@ def bf16_gemm_nt(A, B, D=None, stream=None):
     dev = _one_device(A=A, B=B, D=D)
     with torch.cuda.device(dev):
         _check(lib.bf16_gemm_nt(_ptr(A), _ptr(B), _ptr(D), M, N, K, _stream(stream, dev)), "bf16_gemm_nt")
+    return D
+
+
+def fp8_gemm_nt_ue8m0(A, sfa, B, sfb, D=None, stream=None):
+    """Dense NT GEMM with power-of-two scales: A [M,K] uint8 e4m3, sfa [K/128, ld]
+    uint8 (E8M0: 2^(e-127)), B [N,K] uint8, sfb [ceil(N/128), K/128] uint8 ->
+    D [M,N] bfloat16 (block-scaled tensor-core MMA, FP32 accumulation over K)."""
+    M, K = A.shape
+    N = B.shape[0]
+    _dev(A, torch.uint8, "A"), _dev(B, torch.uint8, "B"), _dev(sfa, torch.uint8, "sfa"), _dev(sfb, torch.uint8, "sfb")
+    if D is None:
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _dev(D, torch.bfloat16, "D")
+    dev = _one_device(A=A, sfa=sfa, B=B, sfb=sfb, D=D)
+    with torch.cuda.device(dev):
+        _check(lib.fp8_gemm_nt_ue8m0(_ptr(A), _ptr(sfa), sfa.shape[1], _ptr(B), _ptr(sfb), _ptr(D), M, N, K,
+                                     _stream(stream, dev)), "fp8_gemm_nt_ue8m0")
     return D

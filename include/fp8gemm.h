@@ -291,6 +291,26 @@ int fp8g_moe_combine(const uint16_t *D, int N, const int32_t *pos, const float *
 int bf16_gemm_nt(const uint16_t *A, const uint16_t *B, uint16_t *D,
                  int M, int N, int K, cudaStream_t stream);
 
+/*
+ * Dense NT GEMM with power-of-two (UE8M0) scales on the block-scaled tensor
+ * cores of the SM100 generation the pages list (kakushin.no, requirements
+ * list: SM90 and SM100):
+ *   D[m,n] = bf16( sum_kb ( sum_{k in kb} A[m,k] * B[n,k] )
+ *                         * 2^(sfa[kb][m] - 127) * 2^(sfb[n/128][kb] - 127) )
+ * with the same 1x128 (A) and 128x128 (B) granularity as fp8_gemm_nt, but
+ * the scales are E8M0 bytes (2^(e-127); 255 would be NaN and must not occur)
+ * applied inside the tensor core, and the whole K sum is accumulated there
+ * in FP32 (no per-K-block promotion), so results differ from fp8_gemm_nt's
+ * within the GEMM tolerance; integer-valued inputs whose sums stay below 2^24
+ * in units of the smallest scale are exact.
+ *   A [M,K] e4m3, sfa [K/128][ld_sf] bytes (ld_sf >= M, ld_sf % 4 == 0),
+ *   B [N,K] e4m3, sfb [ceil(N/128)][K/128] bytes, D [M,N] bf16.
+ * Requirements and conventions otherwise as fp8_gemm_nt.
+ */
+int fp8_gemm_nt_ue8m0(const uint8_t *A, const uint8_t *sfa, int ld_sf,
+                      const uint8_t *B, const uint8_t *sfb,
+                      uint16_t *D, int M, int N, int K, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *fp8g_status_string(int status);
 

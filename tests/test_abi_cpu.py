@@ -123,8 +123,8 @@ def test_every_variant_name_starts_with_its_kind(lib):
     # call's kind; a variant outside the three prefixes would go untested
     names = [lib.fp8g_variant_name(i).decode() for i in range(lib.fp8g_num_variants())]
     for n in names:
-        assert n.split("_", 1)[0] in ("dense", "contiguous", "masked", "bf16"), n
-    for kind in ("dense", "contiguous", "masked", "bf16"):
+        assert n.split("_", 1)[0] in ("dense", "contiguous", "masked", "bf16", "ue8m0"), n
+    for kind in ("dense", "contiguous", "masked", "bf16", "ue8m0"):
         assert any(n.startswith(kind + "_") for n in names), kind
 
 
