@@ -480,7 +480,8 @@ def measure_extras(dev, stream, sampler, steps: int) -> dict:
     """The pieces around the GEMM, each timed in the same run on seeded
     synthetic inputs larger than L2: the FP8 quantisers, the expert dispatch and
     combine of the contiguous layout (a routing of 8192 tokens x top-4 over 4
-    experts, the contiguous workload's 32768 rows) and the BF16 GEMM.  Each
+    experts, the contiguous workload's 32768 rows), the BF16 GEMM and the FP8
+    GEMM with power-of-two scales.  Each
     entry: device time per call (CUDA events over `steps` back-to-back calls
     after warm-up) and its roofline against the measured peaks."""
     import torch
@@ -556,6 +557,23 @@ def measure_extras(dev, stream, sampler, steps: int) -> dict:
         "bound": "tensor", "achieved": tf, "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tf / pk["bf16"],
         "peak_source": f"bf16_tflops (burst) of {pk['source']}"}, "clocks": clk}
     del A, B, Db
+    # FP8 GEMM with power-of-two scales (block-scaled MMA) on the large dense shape
+    M3, N3, K3 = 4096, 7168, 16384
+    A = torch.randint(0, 126, (M3, K3), generator=gen, device=dev, dtype=torch.uint8)
+    B = torch.randint(0, 126, (N3, K3), generator=gen, device=dev, dtype=torch.uint8)
+    sfa = torch.randint(120, 128, (K3 // 128, M3), generator=gen, device=dev, dtype=torch.uint8)
+    sfb = torch.randint(120, 128, ((N3 + 127) // 128, K3 // 128), generator=gen, device=dev, dtype=torch.uint8)
+    D3 = torch.empty(M3, N3, dtype=torch.bfloat16, device=dev)
+    sec, clk = timed(lambda: gemm.fp8_gemm_nt_ue8m0(A, sfa, B, sfb, D3, stream=stream))
+    tf = 2.0 * M3 * N3 * K3 / sec / 1e12
+    peak = pk["bf16"] * FP8_OVER_BF16
+    out["ue8m0_gemm_4096x7168x16384"] = {"what": "FP8 GEMM with power-of-two scales on the block-scaled MMA",
+                                         "us_per_call": sec * 1e6, "variant": gemm.variant_names()[gemm.last_variant()],
+                                         "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                                      "frac": tf / peak, "peak_source":
+                                                      f"bf16_tflops (burst) of {pk['source']} x {FP8_OVER_BF16}"},
+                                         "clocks": clk}
+    del A, B, sfa, sfb, D3
     torch.cuda.empty_cache()
     return out
 

@@ -29,8 +29,9 @@
 //   3 moe_rank_kernel    per chunk: each row's rank among the earlier rows
 //                        of its expert in the chunk (__match_any_sync within
 //                        a warp, per-warp counts across warps), hence pos[r].
-//   4 moe_gather_kernel  one warp per routed row: the token's row quantised
-//                        into row pos[r] of A and its scales (HBM-bound).
+//   4 moe_gather_kernel  one warp per token: the token's row read and
+//                        quantised once, codes and scales stored into every
+//                        row it was routed to (HBM-bound).
 //   5 moe_pad_kernel     zero codes and scales of the padding rows.
 #include <cuda_runtime.h>
 
@@ -136,20 +137,41 @@ __global__ void __launch_bounds__(kChunk) moe_rank_kernel(const int32_t* __restr
   if (r < R) pos[r] = g < 0 ? -1 : off[g] + base[static_cast<long>(blockIdx.x) * G + g] + s_w[w][g] + rank_in_warp;
 }
 
-// One warp per routed row: token t = r / topk quantised into row pos[r].
+// One warp per token: token t is read and quantised once, and its codes and
+// scales are stored into every row pos[t*topk + k] it was routed to (k <
+// topk <= kMaxTopk; dropped slots are skipped).
+constexpr int kMaxTopk = 16;
+
 template <bool kF32>
-__global__ void __launch_bounds__(256, 3) moe_gather_kernel(const void* __restrict__ x, int K, int R, int topk,
+__global__ void __launch_bounds__(256, 3) moe_gather_kernel(const void* __restrict__ x, int K, int T, int topk,
                                                             const int32_t* __restrict__ pos, uint8_t* __restrict__ A,
                                                             float* __restrict__ sa, int ld_sa) {
+  const int lane = threadIdx.x & 31;
   const size_t esz = kF32 ? 4 : 2;
   const long warp = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
-  for (long r = warp; r < R; r += nwarps) {
-    const int p = __ldg(pos + r);
-    if (p < 0) continue;  // warp-uniform
-    const long t = r / topk;
-    quantize_row_1x128<kF32>(static_cast<const uint8_t*>(x) + t * K * esz, K, A + static_cast<long>(p) * K,
-                             [&](int kb, float s) { sa[static_cast<long>(kb) * ld_sa + p] = s; });
+  for (long t = warp; t < T; t += nwarps) {
+    const int mine = lane < topk ? __ldg(pos + t * topk + lane) : -1;
+    int dst[kMaxTopk];
+    bool any = false;
+#pragma unroll
+    for (int k = 0; k < kMaxTopk; ++k) {
+      dst[k] = __shfl_sync(0xffffffffu, mine, k);
+      any = any || (k < topk && dst[k] >= 0);
+    }
+    if (!any) continue;  // warp-uniform
+    quantize_row_1x128<kF32>(
+        static_cast<const uint8_t*>(x) + t * K * esz, K,
+        [&](long off, const auto& c) {
+#pragma unroll
+          for (int k = 0; k < kMaxTopk; ++k)
+            if (k < topk && dst[k] >= 0) store_code_words(A + static_cast<long>(dst[k]) * K + off, c);
+        },
+        [&](int kb, float s) {
+#pragma unroll
+          for (int k = 0; k < kMaxTopk; ++k)
+            if (k < topk && dst[k] >= 0) sa[static_cast<long>(kb) * ld_sa + dst[k]] = s;
+        });
   }
 }
 
@@ -233,7 +255,8 @@ extern "C" int fp8g_moe_dispatch(const void* x, int x_dtype, int T, int K, const
                                  int blocks, uint8_t* A, float* sa, int ld_sa, int32_t* pos, int32_t* m_indices,
                                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (x_dtype != FP8G_IN_BF16 && x_dtype != FP8G_IN_F32) return FP8G_ERR_INVALID_ARG;
-  if (T < 0 || topk < 1 || K <= 0 || K % 128 != 0 || K > 65536 || G < 1 || G > kMaxExperts) return FP8G_ERR_INVALID_ARG;
+  if (T < 0 || topk < 1 || topk > kMaxTopk || K <= 0 || K % 128 != 0 || K > 65536 || G < 1 || G > kMaxExperts)
+    return FP8G_ERR_INVALID_ARG;
   const long R = static_cast<long>(T) * topk;
   if (R > 0x7FFFFFFFL) return FP8G_ERR_INVALID_ARG;
   // capacity for every possible routing: each expert wastes < 128 rows
@@ -256,13 +279,11 @@ extern "C" int fp8g_moe_dispatch(const void* x, int x_dtype, int T, int K, const
   moe_scan_kernel<<<1, kMaxExperts, 0, stream>>>(hist, C, G, off, cnt, m_indices, blocks);
   if (C > 0) {
     moe_rank_kernel<<<C, kChunk, 0, stream>>>(expert, static_cast<int>(R), G, hist, off, pos, err);
-    const long gblocks = std::min<long>((R + 7) / 8, 6L * sms);
+    const long gblocks = std::min<long>((static_cast<long>(T) + 7) / 8, 6L * sms);
     if (x_dtype == FP8G_IN_F32)
-      moe_gather_kernel<true><<<static_cast<unsigned>(gblocks), 256, 0, stream>>>(x, K, static_cast<int>(R), topk, pos,
-                                                                                  A, sa, ld_sa);
+      moe_gather_kernel<true><<<static_cast<unsigned>(gblocks), 256, 0, stream>>>(x, K, T, topk, pos, A, sa, ld_sa);
     else
-      moe_gather_kernel<false><<<static_cast<unsigned>(gblocks), 256, 0, stream>>>(x, K, static_cast<int>(R), topk, pos,
-                                                                                   A, sa, ld_sa);
+      moe_gather_kernel<false><<<static_cast<unsigned>(gblocks), 256, 0, stream>>>(x, K, T, topk, pos, A, sa, ld_sa);
   }
   const long pblocks = std::min<long>((static_cast<long>(G) * 128 + 7) / 8, 4L * sms);
   moe_pad_kernel<<<static_cast<unsigned>(pblocks), 256, 0, stream>>>(off, cnt, G, K, A, sa, ld_sa);

@@ -48,7 +48,8 @@ __global__ void __launch_bounds__(256, 3) quantize_1x128_kernel(const void* __re
   for (long r0 = static_cast<long>(blockIdx.x) * kRowsPerCta; r0 < rows; r0 += static_cast<long>(gridDim.x) * kRowsPerCta) {
     const long row = r0 + w;
     if (row < rows)  // warp-uniform
-      quantize_row_1x128<kF32>(static_cast<const uint8_t*>(x) + row * K * esz, K, q + row * K,
+      quantize_row_1x128<kF32>(static_cast<const uint8_t*>(x) + row * K * esz, K,
+                               [&](long off, const auto& c) { store_code_words(q + row * K + off, c); },
                                [&](int kb, float s) { s_scale[kb][w] = s; });
     __syncthreads();
     // sa[kb][r0 .. r0 + 7]: consecutive threads write consecutive rows

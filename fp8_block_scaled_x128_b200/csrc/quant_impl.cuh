@@ -121,14 +121,16 @@ __device__ __forceinline__ void encode_group(const float (&v)[n], float s, uint3
 }
 
 
-// One row of K elements (K % 128 == 0) quantised per 1x128 group by one warp:
-// codes to q_row, and store_scale(kb, scale) called by one lane per group.
+// One row of K elements (K % 128 == 0) quantised per 1x128 group by one warp.
+// store_codes(offset, c) stores a lane's codes c (kPerLane / 4 words) for the
+// row's elements offset .. offset + kPerLane - 1; store_scale(kb, scale) is
+// called by one lane per group.
 // Every lane loads 16 bytes per step: for bf16 input a half-warp covers one
 // group (8 elements per lane), so a warp step covers two groups of the row;
 // for FP32 input a warp covers one group (4 elements per lane).  kUnits steps
 // (kUnits * 16 bytes per lane) are in flight.  All 32 lanes must call it.
-template <bool kF32, typename StoreScale>
-__device__ __forceinline__ void quantize_row_1x128(const void* __restrict__ x_row, int K, uint8_t* __restrict__ q_row,
+template <bool kF32, typename StoreCodes, typename StoreScale>
+__device__ __forceinline__ void quantize_row_1x128(const void* __restrict__ x_row, int K, StoreCodes store_codes,
                                                    StoreScale store_scale) {
   constexpr int kPerLane = kF32 ? 4 : 8;          // elements per lane per step
   constexpr int kLanesPerGroup = 128 / kPerLane;  // 32 (f32) or 16 (bf16)
@@ -174,15 +176,20 @@ __device__ __forceinline__ void quantize_row_1x128(const void* __restrict__ x_ro
       uint32_t c[kPerLane / 4];
       encode_group(v, sc, c);
       if (kb < KB) {
-        uint8_t* qp = q_row + static_cast<long>(kb) * 128 + l * kPerLane;
-        if constexpr (kF32) {
-          __stcs(reinterpret_cast<uint32_t*>(qp), c[0]);
-        } else {
-          __stcs(reinterpret_cast<uint2*>(qp), make_uint2(c[0], c[1]));
-        }
+        store_codes(static_cast<long>(kb) * 128 + l * kPerLane, c);
         if (l == 0) store_scale(kb, sc);
       }
     }
+  }
+}
+
+// Stores one lane's codes (4 bytes for FP32 input, 8 for bf16) at q.
+template <int n>
+__device__ __forceinline__ void store_code_words(uint8_t* q, const uint32_t (&c)[n]) {
+  if constexpr (n == 1) {
+    __stcs(reinterpret_cast<uint32_t*>(q), c[0]);
+  } else {
+    __stcs(reinterpret_cast<uint2*>(q), make_uint2(c[0], c[1]));
   }
 }
 

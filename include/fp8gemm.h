@@ -249,7 +249,7 @@ size_t fp8g_moe_dispatch_workspace_bytes(int R, int G);
  * Dispatch: builds the contiguous layout and quantises each routed row's
  * token into it, per 1x128 group (as fp8g_quantize_1x128).
  *   x [T][K] (bf16 patterns or FP32, x_dtype), K % 128 == 0, K <= 65536;
- *   expert [T*topk] int32; topk >= 1; 1 <= G <= 256;
+ *   expert [T*topk] int32; 1 <= topk <= 16; 1 <= G <= 256;
  *   blocks >= ceil(T*topk/128) + G (room for any routing);
  *   outputs A [blocks*128][K] e4m3 codes, sa [K/128][ld_sa] (ld_sa >=
  *   blocks*128, ld_sa % 4 == 0), pos [T*topk], m_indices [blocks];
