@@ -129,6 +129,7 @@ struct Params {
 // splitk_reduce_kernel, launched next on the same stream.
 constexpr int kGlobalSplit = -1;
 constexpr int kGlobalSplitPartials = -2;
+
 constexpr int kMaxGSplit = 16;  // the host never picks more
 
 // OPT bits of the promotion (template parameter of both kernels):
@@ -463,12 +464,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
       const uint32_t me = static_cast<uint32_t>(warp - 1);
-      constexpr uint32_t kIdesc = idesc_e4m3_f32(128, BNC);
       uint32_t it = 0;
       bool ok = true;
       for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
         const Tile T = get_tile<kSwap, BNC, KIND, SPLIT>(p, t, rank, false);
         if (!T.valid) continue;
+        // n-lanes: the MMA's N is the tile's rows of A; a masked tail tile
+        // multiplies only its valid rows (rounded up to 16, the MMA's N step)
+        const uint32_t n_mma = kSwap ? static_cast<uint32_t>(min(BNC, (T.mvalid + 15) / 16 * 16)) : BNC;
+        const uint32_t kIdesc = idesc_e4m3_f32(128, n_mma);
         for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
           // stage s and TMEM buffer it % kNBuf (both even counts) belong to
           // issuer s % 2 in every round
@@ -696,6 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (SPLIT == kGlobalSplit) {
     if (warp >= 4) global_split_reduce<BNC, KIND>(p, t_first, rank, abort_flag);
   }
+
   if constexpr (SPLIT > 1) {
     // all partials of this cluster's tile are in place after the barrier;
     // the warpgroup whose columns this CTA owns adds them in rank order
