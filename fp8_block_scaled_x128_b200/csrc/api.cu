@@ -78,9 +78,10 @@ const Variant kVariants[] = {
     make_variant<true, 64, 8, kDense, kGlobalSplitPartials>("dense_nlanes_bn64_st8_gsplit_2k"),
     make_variant<false, 128, 6, kDense, 1>("dense_mlanes_bn128_st6"),
     make_variant<false, 256, 4, kDense, 1>("dense_mlanes_bn256_st4"),
-    make_pair_variant<kDense, 8, 192, kOptFma2>("dense_mlanes_pair_bn192_st8_f"),
+    make_pair_variant<kDense, 6, 192, kOptFma2>("dense_mlanes_pair_bn192_st6_f"),
     make_variant<false, 128, 6, kContiguous, 1>("contiguous_mlanes_bn128_st6"),
     make_variant<false, 256, 4, kContiguous, 1>("contiguous_mlanes_bn256_st4"),
+    make_pair_variant<kContiguous, 6, 192, kOptFma2>("contiguous_mlanes_pair_bn192_st6_f"),
     make_variant<false, 128, 6, kMasked, 1>("masked_mlanes_bn128_st6"),
     make_variant<false, 256, 4, kMasked, 1>("masked_mlanes_bn256_st4"),
     make_pair_variant<kMasked, 6, 192>("masked_mlanes_pair_bn192_st6"),
@@ -98,9 +99,10 @@ enum : int {
   V_DENSE_GSPLIT2K,
   V_DENSE_M128,
   V_DENSE_M256,
-  V_DENSE_PAIR192_S8,
+  V_DENSE_PAIR192,
   V_CONTIG_M128,
   V_CONTIG_M256,
+  V_CONTIG_PAIR192,
   V_MASKED_M128,
   V_MASKED_M256,
   V_MASKED_PAIR192,
@@ -481,7 +483,7 @@ int select_variant(const Problem& P, DeviceInfo* dev, cudaStream_t stream) {
     }
     return V_DENSE_N64;
   }
-  if (pair(V_DENSE_PAIR192_S8, static_cast<long>((P.M + 255) / 256) * ((P.N + 191) / 192))) return V_DENSE_PAIR192_S8;
+  if (pair(V_DENSE_PAIR192, static_cast<long>((P.M + 255) / 256) * ((P.N + 191) / 192))) return V_DENSE_PAIR192;
   return wide(V_DENSE_M256, V_DENSE_M128, static_cast<long>((P.M + 127) / 128) * ((P.N + 255) / 256));
 }
 

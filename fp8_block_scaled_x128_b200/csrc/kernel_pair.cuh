@@ -7,7 +7,10 @@
 //
 //   rank r (0, 1)  holds rows m0 + 128 r .. +127 of A and rows n0 + BN/2 r ..
 //                  + BN/2 - 1 of B for each K-block, in its own shared memory at the
-//                  same offsets as its peer;
+//                  same offsets as its peer, and the 128 values sa[kb][m0 + 128 r ..]
+//                  of its rows (a TMA load of its own, so the promotion reads its
+//                  scales from shared memory: a global load per K-block would wait
+//                  behind the operand stream in the L2-to-SM path);
 //   rank 0         issues tcgen05.mma.cta_group::2 (M = 256, N = BN), which
 //                  reads both CTAs' operands and writes D rows m0 + 128 r of
 //                  all BN columns into CTA r's TMEM;
@@ -19,7 +22,9 @@
 // Barriers (all in each CTA; the ones marked "rank 0" are used there only):
 //   full[s]    rank 0: both CTAs' TMA bytes of stage s (rank 0 posts the
 //              expected count for both)
-//   empty[s]   stage s consumed: one tcgen05.commit multicast to both CTAs
+//   sfull[s]   this CTA's sa slice of stage s
+//   empty[s]   stage s consumed: one tcgen05.commit multicast to both CTAs,
+//              plus one arrival per promotion warp of this CTA (sa slice read)
 //   tfull[b]   partial b ready: one commit multicast to both CTAs
 //   tempty[b]  rank 0: partial b read by the 8 promotion warps of both CTAs
 //              (the peer's arrive remotely)
@@ -61,11 +66,13 @@ template <int STAGES, int BN = 256>
 struct PairLayout {
   static constexpr int kTileBytes = 128 * 128;       // A: 128 rows x one K-block of e4m3
   static constexpr int kBTileBytes = (BN / 2) * 128;  // B: this CTA's BN / 2 rows
+  static constexpr int kSaBytes = 128 * 4;            // sa of this CTA's 128 rows
   static constexpr int kNBuf = 512 / BN >= 4 ? 4 : 2;  // TMEM partial buffers of BN columns
   static constexpr int kOffA = 0;
   static constexpr int kOffB = STAGES * kTileBytes;
-  static constexpr int kOffBar = kOffB + STAGES * kBTileBytes;
-  static constexpr int kNumBars = 2 * STAGES + 2 * kNBuf + 2;
+  static constexpr int kOffSa = kOffB + STAGES * kBTileBytes;
+  static constexpr int kOffBar = kOffSa + STAGES * kSaBytes;
+  static constexpr int kNumBars = 3 * STAGES + 2 * kNBuf + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;
@@ -173,15 +180,19 @@ __global__ void __launch_bounds__(PairShape<BN, NWG>::kThreads, 1)
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + L::kNBuf + b); };
   auto drain_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + 2 * L::kNBuf + i); };
+  auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 * L::kNBuf + 2 + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile uint32_t* abort_flag = tmem_slot + 1;  // [0] abort flag, [1] wait limit (us)
   auto a_tile = [&](int s) { return sbase + L::kOffA + s * L::kTileBytes; };
   auto b_tile = [&](int s) { return sbase + L::kOffB + s * L::kBTileBytes; };
+  auto sa_slot = [&](int s) { return sbase + L::kOffSa + s * L::kSaBytes; };
+  const float* sa_f = reinterpret_cast<const float*>(smem + L::kOffSa);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(empty_bar(s), 1 + 4 * S::kNWG);
+      mbar_init(sfull_bar(s), 1);
     }
     for (int b = 0; b < L::kNBuf; ++b) {
       mbar_init(tfull_bar(b), 1);
@@ -196,6 +207,7 @@ __global__ void __launch_bounds__(PairShape<BN, NWG>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmSA);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), 512);
@@ -244,14 +256,21 @@ __global__ void __launch_bounds__(PairShape<BN, NWG>::kThreads, 1)
             if (rank == 0) mbar_arrive_expect_tx(full_bar(s), kPairStageTx);
             tma_load_3d_pair(a_tile(s), &tmA, fb, kb * 128, arow, ga);
             tma_load_3d_pair(b_tile(s), &tmB, fb, kb * 128, brow, gb);
+            // this CTA's row scales of the K-block (rows past M read as zero)
+            mbar_arrive_expect_tx(sfull_bar(s), L::kSaBytes);
+            tma_load_3d(sa_slot(s), &tmSA, sfull_bar(s), arow, kb, ga);
           }
         }
-        // rank 0 drains: the full barriers count both CTAs' bytes, so every
-        // load of the pair has landed once they complete
-        if (rank == 0) {
+        // drain: rank 0's full barriers count both CTAs' operand bytes, and
+        // each CTA's sfull barriers its own scale loads, so every load of the
+        // pair has landed once they complete
+        {
           const uint32_t first = it > static_cast<uint32_t>(STAGES) ? it - STAGES : 0u;
-          for (uint32_t i = first; i < it; ++i)
-            if ((i % STAGES) % kIssuers == me) drain_phase(full_bar(i % STAGES), (i / STAGES) & 1u);
+          for (uint32_t i = first; i < it; ++i) {
+            if ((i % STAGES) % kIssuers != me) continue;
+            if (rank == 0) drain_phase(full_bar(i % STAGES), (i / STAGES) & 1u);
+            drain_phase(sfull_bar(i % STAGES), (i / STAGES) & 1u);
+          }
         }
       }
     } else if (rank == 0 && lane == 0) {
@@ -314,61 +333,65 @@ __global__ void __launch_bounds__(PairShape<BN, NWG>::kThreads, 1)
       const int nb = min((T.n0 + wg * kCW) / 128, p.NB - 1);
       const float* sbp = p.sb + (static_cast<long>(T.g) * p.NB + nb) * p.KB;
       const bool row_in = m_row < p.M;
-      const float* sap = p.sa + (KIND == kMasked ? static_cast<long>(T.g) * p.KB * p.ld_sa : 0L) + m_row;
-      auto sa_at = [&](int kb) { return row_in && kb < p.KB ? __ldg(sap + static_cast<long>(kb) * p.ld_sa) : 0.f; };
-      auto sb_at = [&](int kb) { return kb < p.KB ? __ldg(sbp + kb) : 0.f; };
-      float sa0 = sa_at(0), sa1 = sa_at(1);
-      float sb0 = sb_at(0), sb1 = sb_at(1);
-      for (int kb = 0; ok && kb < p.KB; kb += 2) {
-        const float sc2[2] = {sa0 * sb0, sa1 * sb1};
-        sa0 = sa_at(kb + 2);
-        sa1 = sa_at(kb + 3);
-        sb0 = sb_at(kb + 2);
-        sb1 = sb_at(kb + 3);
+      // sb of this warpgroup's columns, 32 K-blocks per register: lane i
+      // holds K-block 32 j + i; the next 32 are loaded one chunk ahead and
+      // each K-block's value is broadcast with a shuffle
+      float sb_cur = lane < p.KB ? __ldg(sbp + lane) : 0.f;
+      float sb_nxt = 32 + lane < p.KB ? __ldg(sbp + 32 + lane) : 0.f;
+      for (int kb = 0; ok && kb < p.KB; ++kb, ++it) {
+        if ((kb & 31) == 0 && kb != 0) {
+          sb_cur = sb_nxt;
+          sb_nxt = kb + 32 + lane < p.KB ? __ldg(sbp + kb + 32 + lane) : 0.f;
+        }
+        const float s_b = __shfl_sync(0xffffffffu, sb_cur, kb & 31);
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        const int b = it % L::kNBuf;
+        const uint32_t tph = (it / L::kNBuf) & 1u;
+        bool w = wait_phase(tfull_bar(b), tph, abort_flag);
+        w = w && wait_phase(sfull_bar(s), ph, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // the row's scale for this K-block; the stage's sa slot is free once
+        // every lane has read it (release arrive, after the warp's reads)
+        const float sc = row_in ? sa_f[s * 128 + row] * s_b : 0.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                               static_cast<uint32_t>(b * BNC + wg * kCW);
+        constexpr int kG = S::kGroup;
+        // a CTA whose block belongs to the other expert of this pass only
+        // hands the buffer back
+        if (T.active) {
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (kb + u >= p.KB) break;
-          const int b = it % L::kNBuf;
-          const uint32_t tph = (it / L::kNBuf) & 1u;
-          if (!__all_sync(0xffffffffu, wait_phase(tfull_bar(b), tph, abort_flag))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
-                                 static_cast<uint32_t>(b * BNC + wg * kCW);
-          constexpr int kG = S::kGroup;
-          // a CTA whose block belongs to the other expert of this pass only
-          // hands the buffer back
-          if (T.active) {
+          for (int j0 = 0; j0 < kCW / 32; j0 += kG) {
+            uint32_t r[kG][32];
 #pragma unroll
-            for (int j0 = 0; j0 < kCW / 32; j0 += kG) {
-              uint32_t r[kG][32];
+            for (int j = 0; j < kG; ++j) tmem_ld_32x32b_x32(taddr + 32 * (j0 + j), r[j]);
+            tmem_ld_wait_bind(r[0]);
 #pragma unroll
-              for (int j = 0; j < kG; ++j) tmem_ld_32x32b_x32(taddr + 32 * (j0 + j), r[j]);
-              tmem_ld_wait_bind(r[0]);
+            for (int j = 1; j < kG; ++j) bind_after_wait(r[j]);
 #pragma unroll
-              for (int j = 1; j < kG; ++j) bind_after_wait(r[j]);
+            for (int j = 0; j < kG; ++j) {
+              float* a = acc + 32 * (j0 + j);
+              if constexpr ((OPT & kOptFma2) != 0) {
 #pragma unroll
-              for (int j = 0; j < kG; ++j) {
-                float* a = acc + 32 * (j0 + j);
-                if constexpr ((OPT & kOptFma2) != 0) {
+                for (int c = 0; c < 32; c += 2) ffma2(a[c], a[c + 1], r[j][c], r[j][c + 1], sc);
+              } else {
 #pragma unroll
-                  for (int c = 0; c < 32; c += 2) ffma2(a[c], a[c + 1], r[j][c], r[j][c + 1], sc2[u]);
-                } else {
-#pragma unroll
-                  for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc2[u], a[c]);
-                }
+                for (int c = 0; c < 32; ++c) a[c] = fmaf(__uint_as_float(r[j][c]), sc, a[c]);
               }
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            if (rank == 0) mbar_arrive_relaxed(tempty_bar(b));
-            else mbar_arrive_remote_relaxed(tempty_remote + 8u * b);
-          }
-          ++it;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive_relaxed(tempty_bar(b));
+          else mbar_arrive_remote_relaxed(tempty_remote + 8u * b);
         }
       }
       if (!ok) break;

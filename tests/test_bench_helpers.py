@@ -15,7 +15,7 @@ def test_two_kernel_split_k_counts_both_launches():
     assert bench.kernels_per_call("dense_nlanes_bn64_st8_gsplit_2k") == 2
     assert bench.kernels_per_call("dense_nlanes_bn64_st4_gsplit_2k_x2") == 2
     assert bench.kernels_per_call("dense_nlanes_bn64_st8_gsplit") == 1
-    assert bench.kernels_per_call("dense_mlanes_pair_bn192_st8") == 1
+    assert bench.kernels_per_call("dense_mlanes_pair_bn192_st6_f") == 1
 
 
 def _summary(tmp_path, workload, variant, source_hash, dram):
