@@ -18,10 +18,16 @@
 //                           8 columns in registers, the amax is a CTA max, and
 //                           the codes are stored from the same registers (the
 //                           block is read from HBM once).
+// The 1x128 quantiser (activations, run right before a GEMM) is a programmatic
+// dependent launch: it waits for the previous kernel before it reads x and
+// lets the next kernel (the GEMM) start its prologue, and the early B stream
+// of a GEMM whose B is declared static, at once.
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 
 #include "fp8gemm.h"
 #include "quant_impl.cuh"
@@ -42,6 +48,10 @@ __global__ void __launch_bounds__(256, 3) quantize_1x128_kernel(const void* __re
                                                              uint8_t* __restrict__ q, float* __restrict__ sa,
                                                              int ld_sa) {
   __shared__ float s_scale[kMaxKB][kRowsPerCta];
+  // x may be written by the previous kernel in the stream (a no-op without a
+  // programmatic dependency); the next kernel may start its prologue now
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int w = threadIdx.x >> 5;
   const int KB = K / 128;
   const size_t esz = kF32 ? 4 : 2;
@@ -129,6 +139,33 @@ __global__ void __launch_bounds__(256) quantize_128x128_kernel(const void* __res
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// FP8G_DISABLE_PDL set (and not "0") turns programmatic dependent launch off,
+// as for the GEMMs
+bool pdl_on() {
+  static const bool on = [] {
+    const char* e = std::getenv("FP8G_DISABLE_PDL");
+    return !(e && *e && std::strcmp(e, "0") != 0);
+  }();
+  return on;
+}
+
+template <bool kF32>
+cudaError_t launch_1x128(unsigned blocks, cudaStream_t stream, const void* x, int rows, int K, uint8_t* q, float* sa,
+                         int ld_sa) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(blocks, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  if (pdl_on()) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, quantize_1x128_kernel<kF32>, x, rows, K, q, sa, ld_sa);
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -151,11 +188,13 @@ extern "C" int fp8g_quantize_1x128(const void* x, int x_dtype, int rows, int K, 
   if (K / 128 > kMaxKB) return FP8G_ERR_INVALID_ARG;
   const long row_blocks = (static_cast<long>(rows) + kRowsPerCta - 1) / kRowsPerCta;
   const long blocks = std::min<long>(row_blocks, 16L * sms);
-  if (x_dtype == FP8G_IN_F32)
-    quantize_1x128_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, rows, K, q, sa, ld_sa);
-  else
-    quantize_1x128_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, rows, K, q, sa, ld_sa);
-  if (cudaGetLastError() != cudaSuccess) return FP8G_ERR_CUDA;
+  const cudaError_t e = x_dtype == FP8G_IN_F32
+                            ? launch_1x128<true>(static_cast<unsigned>(blocks), stream, x, rows, K, q, sa, ld_sa)
+                            : launch_1x128<false>(static_cast<unsigned>(blocks), stream, x, rows, K, q, sa, ld_sa);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FP8G_ERR_CUDA;
+  }
   return FP8G_OK;
 }
 

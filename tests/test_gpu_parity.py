@@ -111,6 +111,50 @@ def test_dense_config_64x2112x7168_all_variants(g):
         assert_close(dense_gpu(g, d, v), ex, g.variant_names()[v])
 
 
+@pytest.mark.parametrize("shape", [(1, 8, 128), (65, 200, 256), (257, 520, 256), (64, 2112, 7168)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_dense_after_quantiser_in_one_graph(g, shape):
+    """Quantiser then GEMM, both programmatic dependent launches (the GEMM's
+    prologue may run while the quantiser finishes): in one graph the 1x128
+    quantiser writes A and sa right before each GEMM, alternating between two
+    activations, and every GEMM must use the A written just before it.  Each
+    kernel variant's graph output equals, bit for bit, the same two steps run
+    one call at a time; the quantise-then-GEMM result matches the oracles."""
+    M, N, K = shape
+    d = exact_dense(11, M, N, K)
+    B, sb = dev(d["B"]), dev(d["sb"])
+    gen = torch.Generator(device="cuda").manual_seed(M + N + K)
+    xs = [torch.randn(M, K, device="cuda", generator=gen).to(torch.bfloat16) for _ in range(2)]
+    ld = synth.ld_for(M)
+    A = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    sa = torch.zeros((K // 128, ld), dtype=torch.float32, device="cuda")
+    q0, sa0 = oracle.quantize_1x128(xs[0].float().cpu().numpy(), ld_sa=ld)
+    ex, _ = oracle.gemm_nt(q0, sa0, ld, d["B"], d["sb"], M, N, K)
+    for v in variants(g, "dense_"):
+        g.set_variant_override(v)
+        try:
+            refs = []
+            for x in xs:
+                g.quantize_1x128(x, q=A, sa=sa, ld_sa=ld)
+                refs.append(host_bits(g.fp8_gemm_nt(A, sa, B, sb)))
+            assert_close(refs[0], ex, f"{g.variant_names()[v]} {shape}")
+            outs = [canary_like((M, N)) for _ in range(4)]
+            stream = torch.cuda.Stream()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                for i in range(4):
+                    g.quantize_1x128(xs[i % 2], q=A, sa=sa, ld_sa=ld, stream=stream)
+                    g.fp8_gemm_nt(A, sa, B, sb, D=outs[i], stream=stream)
+            graph.replay()
+            torch.cuda.synchronize()
+            for i in range(4):
+                assert np.array_equal(host_bits(outs[i]), refs[i % 2]), (g.variant_names()[v], i)
+            del graph
+        finally:
+            g.set_variant_override(None)
+    assert g.device_error() == 0
+
+
 def test_dense_is_deterministic(g):
     d = synth.config_inputs("dense_64x2112x7168")
     first = dense_gpu(g, d)
