@@ -36,14 +36,16 @@ struct Variant {
   bool pair;        // CTA pairs (clusters of two) sharing a 256 x bnc tile
   int threads;      // threads per CTA
   int launch_regs;  // register-split variants: registers per thread at launch
+  bool tma_store = false;  // m-lanes TMA-store epilogue: the third tensor map is D
 };
 
 template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int OPT = 0>
 Variant make_variant(const char* name) {
-  using L = Layout<kSwap, BNC, STAGES, SPLIT>;
-  return Variant{name, KIND, kSwap, BNC, STAGES, SPLIT, L::kRegSplit,
+  constexpr bool kStore = (OPT & kOptTmaStore) != 0;
+  using L = Layout<kSwap, BNC, STAGES, SPLIT, kStore>;
+  return Variant{name,     KIND, kSwap, BNC, STAGES, SPLIT, L::kRegSplit,
                  &fp8_gemm_kernel<kSwap, BNC, STAGES, KIND, SPLIT, OPT>, L::kSmemAlloc, false,
-                 kThreads, kLaunchRegs};
+                 kThreads, kLaunchRegs, kStore};
 }
 
 template <int STAGES, bool kTmaStore>
@@ -81,7 +83,7 @@ const Variant kVariants[] = {
     make_pair_variant<kDense, 6, 192, kOptFma2>("dense_mlanes_pair_bn192_st6_f"),
     make_variant<false, 128, 6, kContiguous, 1>("contiguous_mlanes_bn128_st6"),
     make_variant<false, 256, 4, kContiguous, 1>("contiguous_mlanes_bn256_st4"),
-    make_pair_variant<kContiguous, 6, 192, kOptFma2>("contiguous_mlanes_pair_bn192_st6_f"),
+    make_variant<false, 256, 4, kContiguous, 1, kOptTmaStore>("contiguous_mlanes_bn256_st4_tmastore"),
     make_variant<false, 128, 6, kMasked, 1>("masked_mlanes_bn128_st6"),
     make_variant<false, 256, 4, kMasked, 1>("masked_mlanes_bn256_st4"),
     make_pair_variant<kMasked, 6, 192>("masked_mlanes_pair_bn192_st6"),
@@ -102,7 +104,7 @@ enum : int {
   V_DENSE_PAIR192,
   V_CONTIG_M128,
   V_CONTIG_M256,
-  V_CONTIG_PAIR192,
+  V_CONTIG_M256_TMASTORE,
   V_MASKED_M128,
   V_MASKED_M256,
   V_MASKED_PAIR192,
@@ -366,7 +368,11 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
   if (!rc)
     rc = encode3d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, P.B, P.K, P.N, G_b, (uint64_t)P.K,
                   (uint64_t)P.K * P.N, 128, b_box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!rc)
+  if (!rc && V.tma_store)
+    // the third map is D: boxes of 32 rows x 32 columns (clipped at M and N)
+    rc = encode3d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P.D, P.N, P.M, 1, (uint64_t)P.N * 2,
+                  (uint64_t)P.N * 2 * P.M, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else if (!rc)
     rc = encode3d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, P.sa, P.M, KB, G_a, (uint64_t)P.ld_sa * 4,
                   (uint64_t)P.ld_sa * 4 * KB, V.swap ? V.bnc : 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
@@ -447,12 +453,15 @@ int select_variant(const Problem& P, DeviceInfo* dev, cudaStream_t stream) {
   auto pair = [&](int v, long pair_tiles) {
     return prepare_variant(dev, v) == FP8G_OK && dev->max_clusters[v] > 0 && pair_tiles >= dev->max_clusters[v];
   };
-  // contiguous: the pair variant is correct for any expert layout (a pair
-  // tile that straddles two experts runs once per expert) but measured
-  // slower than the single-CTA tiles on G=4, M=8192 per expert, N=4096,
-  // K=7168 (1295 vs 1257 us), so it is only reached by an explicit choice
-  if (P.kind == kContiguous)
-    return wide(V_CONTIG_M256, V_CONTIG_M128, static_cast<long>(P.M / 128) * ((P.N + 255) / 256));
+  // contiguous: single-CTA 128 x 256 tiles with the TMA-store epilogue
+  // (G=4, M=8192 per expert, N=4096, K=7168: 1212-1227 us against 1243-1245
+  // us with direct stores; CTA pairs with 256 x 192 tiles 1317-1345 us, 256 x
+  // 256 pair tiles 1401 us); direct stores if its shared memory cannot be had
+  if (P.kind == kContiguous) {
+    const long tiles256 = static_cast<long>(P.M / 128) * ((P.N + 255) / 256);
+    if (tiles256 >= dev->sms && prepare_variant(dev, V_CONTIG_M256_TMASTORE) == FP8G_OK) return V_CONTIG_M256_TMASTORE;
+    return wide(V_CONTIG_M256, V_CONTIG_M128, tiles256);
+  }
   if (P.kind == kMasked) {
     // B streams once per 128 (or 256) rows of a group's A: m-lanes tiles read
     // it the fewest times; count the tiles the typical group fills

@@ -139,6 +139,14 @@ constexpr int kMaxGSplit = 16;  // the host never picks more
 //             slower on the single-CTA 256-wide kernel, whose promotion
 //             threads then spill.
 constexpr int kOptFma2 = 2;
+//   kOptTmaStore (m-lanes, single CTA, no split): the epilogue stages each
+//             warp's 32 rows x 32 columns of bf16 in shared memory (two
+//             buffers per warp) and one lane stores them with a TMA tensor
+//             store; the D tensor map takes the third map slot (tmSA, which
+//             the m-lanes kernels do not use otherwise).  Every row of a
+//             valid tile is written (contiguous and dense tiles, whose rows
+//             past M the map clips), so masked tiles keep direct stores.
+constexpr int kOptTmaStore = 4;
 
 constexpr int pow2_at_least(int x, int lo) {
   int p = lo;
@@ -146,7 +154,7 @@ constexpr int pow2_at_least(int x, int lo) {
   return p;
 }
 
-template <bool kSwap, int BNC, int STAGES, int SPLIT>
+template <bool kSwap, int BNC, int STAGES, int SPLIT, bool kTmaStore = false>
 struct Layout {
   static constexpr int kLaneBytes = 128 * 128;   // 128 rows x 128 e4m3 (one K-block)
   static constexpr int kColBytes = BNC * 128;
@@ -161,7 +169,10 @@ struct Layout {
   static constexpr int kOffSa = kOffCol + STAGES * kColBytes;
   static constexpr int kOffRecv = kOffSa + STAGES * kSaFloats * 4;
   static constexpr int kRecvBytes = SPLIT > 1 ? SPLIT * 128 * kCPD * 4 : 0;
-  static constexpr int kOffBar = kOffRecv + kRecvBytes;
+  static constexpr int kStoreChunk = 32 * 32 * 2;                       // one warp's 32 x 32 bf16
+  static constexpr int kOffStore = kOffRecv + kRecvBytes;
+  static constexpr int kStoreBytes = kTmaStore ? 8 * 2 * kStoreChunk : 0;  // 8 promotion warps x 2 buffers
+  static constexpr int kOffBar = kOffStore + kStoreBytes;
   static constexpr int kNumBars = 2 * STAGES + 2 * kNBuf + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
@@ -179,6 +190,7 @@ struct Layout {
   static_assert(!kRegSplit || !kSwap, "the register split is for the m-lanes orientation");
   static_assert(kSmemAlloc <= 232448, "shared memory");
   static_assert(kNBuf >= 2, "TMEM buffers");
+  static_assert(!kTmaStore || (!kSwap && SPLIT == 1), "TMA-store epilogue: m-lanes tiles without split-K");
 };
 
 // Register budget of the BNC = 256 variants: 384 threads launch with 168
@@ -348,7 +360,9 @@ template <bool kSwap, int BNC, int STAGES, int KIND, int SPLIT, int OPT = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSA, const Params p) {
-  using L = Layout<kSwap, BNC, STAGES, SPLIT>;
+  constexpr bool kTmaStore = (OPT & kOptTmaStore) != 0;
+  using L = Layout<kSwap, BNC, STAGES, SPLIT, kTmaStore>;
+  static_assert(!kTmaStore || KIND != kMasked, "masked tiles store only their valid rows");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -513,6 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = 32 * q + lane;  // tile row = TMEM lane
     float acc[kCW];
     uint32_t it = 0;
+    [[maybe_unused]] uint32_t store_it = 0;  // TMA-store epilogue: chunks stored by this warp
     bool ok = true;
     for (int t = t_first; ok && t < p.num_tiles; t += t_step) {
       // one thread records bad m_indices / masked_m entries in the error word
@@ -676,6 +691,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kCW; ++c)
             if (c < live) dcol[static_cast<long>(c) * p.N] = static_cast<uint16_t>(pack_bf16x2(acc[c], 0.f) & 0xFFFFu);
         }
+      } else if constexpr (kTmaStore) {
+        // a warp's 32 rows x 32 columns at a time through shared memory; the
+        // store issued from the other buffer may still be reading it: wait
+        // for all but the latest group before overwriting
+        const CUtensorMap* tmD = &tmSA;
+        const uint32_t stage0 = sbase + L::kOffStore + static_cast<uint32_t>((warp - 4) * 2 * L::kStoreChunk);
+#pragma unroll
+        for (int c0 = 0; c0 < kCW; c0 += 32) {
+          const uint32_t buf = stage0 + (store_it & 1u) * L::kStoreChunk;
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 v;
+            v.x = pack_bf16x2(acc[c0 + 8 * j + 0], acc[c0 + 8 * j + 1]);
+            v.y = pack_bf16x2(acc[c0 + 8 * j + 2], acc[c0 + 8 * j + 3]);
+            v.z = pack_bf16x2(acc[c0 + 8 * j + 4], acc[c0 + 8 * j + 5]);
+            v.w = pack_bf16x2(acc[c0 + 8 * j + 6], acc[c0 + 8 * j + 7]);
+            st_shared_v4(buf + static_cast<uint32_t>(lane * 64 + j * 16), v);
+          }
+          fence_proxy_async_shared();
+          __syncwarp();
+          const int n = T.n0 + wg * kCW + c0;
+          if (lane == 0 && n < p.N) {
+            tma_store_3d(tmD, buf, n, T.m0 + 32 * q, 0);
+            bulk_commit_group();
+          }
+          ++store_it;
+        }
       } else {
         // a thread holds kCW consecutive columns of its row: 16-byte stores
         if (row < T.mvalid) {
@@ -693,6 +737,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+    }
+    if constexpr (kTmaStore) {
+      // every store of this warp has finished (its shared memory may go)
+      if (lane == 0) bulk_wait_group<0>();
+      __syncwarp();
     }
   }
 
