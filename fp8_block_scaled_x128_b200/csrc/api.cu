@@ -86,7 +86,7 @@ const Variant kVariants[] = {
     make_variant<false, 256, 4, kContiguous, 1, kOptTmaStore>("contiguous_mlanes_bn256_st4_tmastore"),
     make_variant<false, 128, 6, kMasked, 1>("masked_mlanes_bn128_st6"),
     make_variant<false, 256, 4, kMasked, 1>("masked_mlanes_bn256_st4"),
-    make_pair_variant<kMasked, 6, 192>("masked_mlanes_pair_bn192_st6"),
+    make_pair_variant<kMasked, 6, 192, kOptFma2>("masked_mlanes_pair_bn192_st6_f"),
     make_bf16_variant<6, false>("bf16_pair_bn256_st6"),
     make_bf16_variant<6, true>("bf16_pair_bn256_st6_tmastore"),
     make_ue8m0_variant<4>("ue8m0_mlanes_bn256_st4"),

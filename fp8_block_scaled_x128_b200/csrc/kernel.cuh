@@ -134,10 +134,10 @@ constexpr int kMaxGSplit = 16;  // the host never picks more
 
 // OPT bits of the promotion (template parameter of both kernels):
 //   kOptFma2: packed FP32x2 fused multiply-adds (fma.rn.f32x2; each half
-//             rounds like fmaf, so results are unchanged).  Measured on the
-//             large dense shape: 5-11 % fewer cycles on the CTA-pair kernel;
-//             slower on the single-CTA 256-wide kernel, whose promotion
-//             threads then spill.
+//             rounds like fmaf, so results are unchanged).  Measured: 5-11 %
+//             fewer cycles on the dense CTA-pair kernel, 4-5 % less time on
+//             the masked one; slower on the single-CTA 256-wide kernel, whose
+//             promotion threads then spill.
 constexpr int kOptFma2 = 2;
 //   kOptTmaStore (m-lanes, single CTA, no split): the epilogue stages each
 //             warp's 32 rows x 32 columns of bf16 in shared memory (two
