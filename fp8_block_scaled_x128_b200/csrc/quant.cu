@@ -10,8 +10,8 @@
 //   code  = e4m3_rne_satfinite(x / scale)   (one IEEE FP32 division)
 //
 // Both kernels are HBM-bound streams: each input element is read once (2 or
-// 4 bytes) and each code written once (1 byte).  The arithmetic (and the
-// division-free exact quotient test) is in quant_impl.cuh.
+// 4 bytes) and each code written once (1 byte).  The arithmetic (the
+// correctly rounded quotient without a division) is in quant_impl.cuh.
 //   quantize_1x128_kernel   a warp per row (quantize_row_1x128), 8 rows per
 //                           CTA, scales staged in shared memory.
 //   quantize_128x128_kernel one CTA per 128x128 block: a thread holds 8 rows x
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(256) quantize_128x128_kernel(const void* __res
     float v[8];
     values(i, v);
     uint32_t c[2];
-    encode_group(v, s, c);  // every lane takes part (the rare exact branch is a warp vote)
+    encode_group(v, s, c);
     if (r < N) __stcs(reinterpret_cast<uint2*>(q + static_cast<long>(r) * K + c0), make_uint2(c[0], c[1]));
   }
   if (t == 0) sb[static_cast<long>(nb) * KB + kb] = s;

@@ -6,16 +6,11 @@
 //   code  = e4m3_rne_satfinite(x / scale)   (one IEEE FP32 division)
 //
 // The division.  A full IEEE division per element would make the kernels
-// ALU-bound.  Only the e4m3 code of the quotient matters, and that code
-// changes only where the quotient crosses a rounding midpoint between two
-// e4m3 values.  So each element first takes q0 = x * r with r the correctly
-// rounded reciprocal of the group's scale: q0 is within 2.5 FP32 ulps of the
-// correctly rounded quotient fl(x / s).  When q0 lies more than 8 ulps from
-// every e4m3 midpoint, both round to the same code and q0 is used; otherwise
-// an exact test decides on which side of the midpoint fl(x / s) lies
-// (midpoint_side, no division).  bf16 inputs put about 0.5 % of quotients on
-// or next to a midpoint.  The codes are therefore those of e4m3(fl(x / s)),
-// bit for bit.
+// ALU-bound.  Each element instead takes the product with the correctly
+// rounded reciprocal of the group's scale and two Markstein correction steps
+// (quotient_rn: one multiply and four FMAs, no branch), which give the
+// correctly rounded quotient fl(x / s); its e4m3 conversion is then exactly
+// the code of the definition, bit for bit.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -31,90 +26,46 @@ constexpr int kUnits = 8;  // 16-byte loads per lane in flight per warp
 
 __device__ __forceinline__ float scale_of(float amax) { return amax > 0.f ? __fdiv_rn(amax, kE4M3Max) : 1.f; }
 
-// True when q0 is more than 8 ulps away from every rounding midpoint of e4m3
-// (normal range |q0| >= 2^-6: the midpoint sits where the 20 mantissa bits
-// below e4m3's 3 are 0x80000; subnormal range: quantum 2^-9, midpoints at odd
-// multiples of 2^-10, checked on |q0| * 512 with a margin of 2^-17).
-__device__ __forceinline__ bool far_from_midpoint(float q0) {
-  const uint32_t a = __float_as_uint(q0) & 0x7FFFFFFFu;
-  if (a >= 0x3C800000u) {  // 2^-6
-    const int low = static_cast<int>(a & 0xFFFFFu) - 0x80000;
-    return low > 8 || low < -8;
-  }
-  const float t = __uint_as_float(a) * 512.f;
-  const float d = t - floorf(t) - 0.5f;
-  return fabsf(d) > 7.62939453e-06f;  // 2^-17
-}
-
 // Two floats -> two e4m3 codes (round to nearest even, saturating at +-448),
 // lo in the low byte.
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
-// For a quotient near an e4m3 rounding midpoint: a value that converts to the
-// same e4m3 code as fl(x / s).  q0 = x * r lies within 2.5 ulps of fl(x / s)
-// and within 8 ulps of the midpoint m nearest to it.  m has at most 5
-// significant bits, so d = x - m * s is a multiple of 2^(e_m + e_s - 27) of
-// at most 9 bits and the FMA computes it exactly; with s > 0,
-//   |d| <= ulp(m)/2 * s  <=>  fl(x / s) == m  (m's last bit is even, so a tie
-//                              of the FP32 rounding also lands on m),
-//   d > ulp(m)/2 * s     <=>  fl(x / s) lies above m,  d < -... below it.
-// On m itself the conversion breaks the e4m3 tie to even; off it, the next
-// float on the correct side of m converts to the correct neighbour.
-__device__ __forceinline__ float midpoint_side(float x, float s, float q0) {
-  const uint32_t sign = __float_as_uint(q0) & 0x80000000u;
-  const uint32_t a = __float_as_uint(q0) & 0x7FFFFFFFu;
-  uint32_t mb;  // |m|
-  if (a >= 0x3C800000u) {
-    mb = (a & 0xFFF00000u) | 0x00080000u;  // keep exponent and 3 mantissa bits, set the half bit
-  } else {
-    const float t = __uint_as_float(a) * 512.f;
-    mb = __float_as_uint((floorf(t) + 0.5f) * 0.001953125f);  // (k + 1/2) * 2^-9
-  }
-  const float m = __uint_as_float(mb | sign);
-  const float d = fmaf(-m, s, x);
-  const float half_ulp = __uint_as_float(((mb >> 23) - 24u) << 23);  // 2^(e_m - 24)
-  const float lim = half_ulp * s;
-  if (fabsf(d) <= lim) return m;
-  return __uint_as_float((d > 0.f) == (sign == 0u) ? (mb + 1u) | sign : (mb - 1u) | sign);
+// fl(x / s), the correctly rounded binary32 quotient, without a division:
+// Markstein's correction step (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34,
+// 1990; the division theorem as stated in Muller et al., Handbook of
+// Floating-Point Arithmetic): with y = RN(1/s) and an approximation q within
+// one ulp of x / s, the residual x - s q is exact in one FMA and
+// RN(q + (x - s q) y) = RN(x / s).  q0 = RN(x y) can be up to 1.5 ulps off,
+// so one correction brings it within one ulp (0.5 ulp plus 2^-23 ulp) and a
+// second gives the correctly rounded quotient.  Valid while x / s and the
+// residuals stay normal or zero: |x| <= 448.1 s and s is at least 2^-90 here
+// (encode_group scales smaller groups up), so the quotient never overflows,
+// and a quotient below 2^-126 is far under e4m3's smallest rounding boundary
+// (2^-10), where only its sign matters (restored from x, so -0 stays -0).
+__device__ __forceinline__ float quotient_rn(float x, float s, float y) {
+  float q = x * y;
+  q = fmaf(fmaf(-q, s, x), y, q);
+  q = fmaf(fmaf(-q, s, x), y, q);
+  return copysignf(q, x);
 }
 
 // Codes of n values of one group with scale s, packed 4 per 32-bit word
-// (lowest element in the lowest byte).  Each value takes the fast quotient
-// q0 = x * r (r = 1/s correctly rounded); the few that lie near an e4m3
-// midpoint are settled by midpoint_side, one per lane and loop trip, so the
-// code for them exists once.  A group with a scale below 2^-90 is first
-// scaled by 2^100 together with its values (exact), so that the reciprocal
-// and the midpoint test stay in the normal range; no scale can exceed
-// FLT_MAX / 448, so no group needs the opposite.  Every lane of the warp must
-// call it (the loop runs while any lane has work).
+// (lowest element in the lowest byte): e4m3(fl(x / s)) for every value, from
+// the correctly rounded quotient above.  A group with a scale below 2^-90 is
+// first scaled by 2^100 together with its values (exact), so that the
+// reciprocal and the residuals stay in the normal range; no scale can exceed
+// FLT_MAX / 448, so no group needs the opposite.
 template <int n>
 __device__ __forceinline__ void encode_group(const float (&v)[n], float s, uint32_t (&c)[n / 4]) {
   const float k = s < 8.07793567e-28f ? 1.26765060e30f : 1.f;  // 2^-90, 2^100
   const float ss = s * k;
-  const float r = __frcp_rn(ss);
+  const float y = __frcp_rn(ss);
   float qv[n];
-  uint32_t near = 0u;
 #pragma unroll
-  for (int i = 0; i < n; ++i) {
-    qv[i] = (v[i] * k) * r;
-    if (!far_from_midpoint(qv[i])) near |= 1u << i;
-  }
-  while (__any_sync(0xffffffffu, near != 0u)) {
-    const int idx = near != 0u ? __ffs(near) - 1 : 0;
-    float xi = v[0], qi = qv[0];
-#pragma unroll
-    for (int j = 1; j < n; ++j)
-      if (idx == j) xi = v[j], qi = qv[j];
-    const float fixed = midpoint_side(xi * k, ss, qi);
-    if (near != 0u) {
-#pragma unroll
-      for (int j = 0; j < n; ++j)
-        if (idx == j) qv[j] = fixed;
-    }
-    near &= near - 1u;
-  }
+  for (int i = 0; i < n; ++i) qv[i] = quotient_rn(v[i] * k, ss, y);
 #pragma unroll
   for (int i = 0; i < n / 4; ++i)
     c[i] = e4m3x2(qv[4 * i], qv[4 * i + 1]) | (e4m3x2(qv[4 * i + 2], qv[4 * i + 3]) << 16);
