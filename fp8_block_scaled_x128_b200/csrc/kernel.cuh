@@ -692,13 +692,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c < live) dcol[static_cast<long>(c) * p.N] = static_cast<uint16_t>(pack_bf16x2(acc[c], 0.f) & 0xFFFFu);
         }
       } else if constexpr (kTmaStore) {
-        // a warp's 32 rows x 32 columns at a time through shared memory; the
-        // store issued from the other buffer may still be reading it: wait
-        // for all but the latest group before overwriting
+        // a warp's 32 rows x 32 columns at a time through shared memory, for
+        // the chunks inside D (warp-uniform): every buffer write is followed
+        // by a store, so waiting until at most one store group is pending
+        // (the other buffer's) frees the buffer about to be written
         const CUtensorMap* tmD = &tmSA;
         const uint32_t stage0 = sbase + L::kOffStore + static_cast<uint32_t>((warp - 4) * 2 * L::kStoreChunk);
 #pragma unroll
         for (int c0 = 0; c0 < kCW; c0 += 32) {
+          const int n = T.n0 + wg * kCW + c0;
+          if (n >= p.N) continue;
           const uint32_t buf = stage0 + (store_it & 1u) * L::kStoreChunk;
           if (lane == 0) bulk_wait_group_read<1>();
           __syncwarp();
@@ -713,8 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_shared();
           __syncwarp();
-          const int n = T.n0 + wg * kCW + c0;
-          if (lane == 0 && n < p.N) {
+          if (lane == 0) {
             tma_store_3d(tmD, buf, n, T.m0 + 32 * q, 0);
             bulk_commit_group();
           }

@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kBf16Threads, 1)
       const int m = T.m0 + 128 * static_cast<int>(rank) + row;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * BN);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32, ++chunk_it) {
+      for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(taddr + c0, r);
         tmem_ld_wait_bind(r);
@@ -209,18 +209,24 @@ __global__ void __launch_bounds__(kBf16Threads, 1)
         }
         const int n = T.n0 + c0;
         if constexpr (kTmaStore) {
-          // this warp's 32 rows x 32 columns through shared memory; a store
-          // of the other buffer may still be reading: wait for all but one
-          const uint32_t buf_addr = stage0 + (chunk_it & 1u) * L::kStageBytes;
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
+          // this warp's 32 rows x 32 columns through shared memory, if any of
+          // them is inside D (warp-uniform): every buffer write is followed
+          // by a store, so waiting until at most one store group is pending
+          // (the other buffer's) frees this buffer
+          const int r0 = T.m0 + 128 * static_cast<int>(rank) + 32 * q;
+          if (n < p.N && r0 < p.M) {
+            const uint32_t buf_addr = stage0 + (chunk_it & 1u) * L::kStageBytes;
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) st_shared_v4(buf_addr + static_cast<uint32_t>(lane * 64 + j * 16), v[j]);
-          fence_proxy_async_shared();
-          __syncwarp();
-          if (lane == 0 && n < p.N && T.m0 + 128 * static_cast<int>(rank) + 32 * q < p.M) {
-            tma_store_3d(&tmD, buf_addr, n, T.m0 + 128 * static_cast<int>(rank) + 32 * q, 0);
-            bulk_commit_group();
+            for (int j = 0; j < 4; ++j) st_shared_v4(buf_addr + static_cast<uint32_t>(lane * 64 + j * 16), v[j]);
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tmD, buf_addr, n, r0, 0);
+              bulk_commit_group();
+            }
+            ++chunk_it;
           }
         } else {
           if (m < p.M) {
