@@ -26,7 +26,7 @@
 //   empty[s]   stage s consumed: one tcgen05.commit multicast to both CTAs,
 //              plus one arrival per promotion warp of this CTA (sa slice read)
 //   tfull[b]   partial b ready: one commit multicast to both CTAs
-//   tempty[b]  rank 0: partial b read by the 8 promotion warps of both CTAs
+//   tempty[b]  rank 0: partial b read by every promotion warp of both CTAs
 //              (the peer's arrive remotely)
 // Every wait is bounded as in fp8_gemm_kernel; the CTAs of a pair leave
 // through one cluster barrier after all their work (and aborts) have drained.

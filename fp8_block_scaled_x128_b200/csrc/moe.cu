@@ -142,7 +142,9 @@ __global__ void __launch_bounds__(kChunk) moe_rank_kernel(const int32_t* __restr
 // topk <= kMaxTopk; dropped slots are skipped).
 constexpr int kMaxTopk = 16;
 
-template <bool kF32>
+// kCap: a compile-time bound on topk (4, 8 or 16, the smallest that holds
+// it), so each store of a lane's codes tests only that many destinations
+template <bool kF32, int kCap>
 __global__ void __launch_bounds__(256, 3) moe_gather_kernel(const void* __restrict__ x, int K, int T, int topk,
                                                             const int32_t* __restrict__ pos, uint8_t* __restrict__ A,
                                                             float* __restrict__ sa, int ld_sa) {
@@ -152,10 +154,10 @@ __global__ void __launch_bounds__(256, 3) moe_gather_kernel(const void* __restri
   const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
   for (long t = warp; t < T; t += nwarps) {
     const int mine = lane < topk ? __ldg(pos + t * topk + lane) : -1;
-    int dst[kMaxTopk];
+    int dst[kCap];
     bool any = false;
 #pragma unroll
-    for (int k = 0; k < kMaxTopk; ++k) {
+    for (int k = 0; k < kCap; ++k) {
       dst[k] = __shfl_sync(0xffffffffu, mine, k);
       any = any || (k < topk && dst[k] >= 0);
     }
@@ -164,12 +166,12 @@ __global__ void __launch_bounds__(256, 3) moe_gather_kernel(const void* __restri
         static_cast<const uint8_t*>(x) + t * K * esz, K,
         [&](long off, const auto& c) {
 #pragma unroll
-          for (int k = 0; k < kMaxTopk; ++k)
+          for (int k = 0; k < kCap; ++k)
             if (k < topk && dst[k] >= 0) store_code_words(A + static_cast<long>(dst[k]) * K + off, c);
         },
         [&](int kb, float s) {
 #pragma unroll
-          for (int k = 0; k < kMaxTopk; ++k)
+          for (int k = 0; k < kCap; ++k)
             if (k < topk && dst[k] >= 0) sa[static_cast<long>(kb) * ld_sa + dst[k]] = s;
         });
   }
@@ -280,10 +282,18 @@ extern "C" int fp8g_moe_dispatch(const void* x, int x_dtype, int T, int K, const
   if (C > 0) {
     moe_rank_kernel<<<C, kChunk, 0, stream>>>(expert, static_cast<int>(R), G, hist, off, pos, err);
     const long gblocks = std::min<long>((static_cast<long>(T) + 7) / 8, 6L * sms);
-    if (x_dtype == FP8G_IN_F32)
-      moe_gather_kernel<true><<<static_cast<unsigned>(gblocks), 256, 0, stream>>>(x, K, T, topk, pos, A, sa, ld_sa);
-    else
-      moe_gather_kernel<false><<<static_cast<unsigned>(gblocks), 256, 0, stream>>>(x, K, T, topk, pos, A, sa, ld_sa);
+    const unsigned gb = static_cast<unsigned>(gblocks);
+    const bool f32 = x_dtype == FP8G_IN_F32;
+    if (topk <= 4) {
+      if (f32) moe_gather_kernel<true, 4><<<gb, 256, 0, stream>>>(x, K, T, topk, pos, A, sa, ld_sa);
+      else moe_gather_kernel<false, 4><<<gb, 256, 0, stream>>>(x, K, T, topk, pos, A, sa, ld_sa);
+    } else if (topk <= 8) {
+      if (f32) moe_gather_kernel<true, 8><<<gb, 256, 0, stream>>>(x, K, T, topk, pos, A, sa, ld_sa);
+      else moe_gather_kernel<false, 8><<<gb, 256, 0, stream>>>(x, K, T, topk, pos, A, sa, ld_sa);
+    } else {
+      if (f32) moe_gather_kernel<true, kMaxTopk><<<gb, 256, 0, stream>>>(x, K, T, topk, pos, A, sa, ld_sa);
+      else moe_gather_kernel<false, kMaxTopk><<<gb, 256, 0, stream>>>(x, K, T, topk, pos, A, sa, ld_sa);
+    }
   }
   const long pblocks = std::min<long>((static_cast<long>(G) * 128 + 7) / 8, 4L * sms);
   moe_pad_kernel<<<static_cast<unsigned>(pblocks), 256, 0, stream>>>(off, cnt, G, K, A, sa, ld_sa);

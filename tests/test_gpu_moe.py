@@ -63,7 +63,8 @@ def check_dispatch(g, x, e, topk, G, dtype="bf16"):
 
 
 @pytest.mark.parametrize("T,topk,G,K,drop", [(300, 2, 5, 384, 0.0), (4096, 8, 64, 1024, 0.05), (1, 1, 1, 128, 0.0),
-                                             (2500, 6, 256, 256, 0.0), (129, 3, 7, 7168, 0.2)])
+                                             (2500, 6, 256, 256, 0.0), (129, 3, 7, 7168, 0.2),
+                                             (200, 12, 16, 256, 0.1)])
 def test_dispatch_matches_oracle(g, T, topk, G, K, drop):
     check_dispatch(g, tokens(T + K, T, K), routing(T + G, T, topk, G, drop), topk, G)
     assert g.device_error() == 0
