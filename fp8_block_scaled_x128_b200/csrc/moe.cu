@@ -198,40 +198,51 @@ __global__ void __launch_bounds__(256) moe_pad_kernel(const int32_t* __restrict_
   }
 }
 
-// out[t, 8j .. 8j+7] from the topk rows pos[t*topk + k] of D: one thread per
-// (token, 8 columns), 16-byte loads and stores.
+// out[t, 8j .. 8j+7] from the topk rows pos[t*topk + k] of D: a CTA per
+// token (grid-stride), its threads over the 16-byte column groups j.  The
+// token's slots (positions and weights, kCap >= topk of them) are read once;
+// all of a thread's row loads are issued before the first FMA, and the FMAs
+// run in slot order, one rounding each, as the definition states.
+template <int kCap>
 __global__ void __launch_bounds__(256) moe_combine_kernel(const uint16_t* __restrict__ D, int N,
                                                           const int32_t* __restrict__ pos, const float* __restrict__ w,
                                                           int T, int topk, uint16_t* __restrict__ out) {
   const int per_row = N / 8;
-  const long items = static_cast<long>(T) * per_row;
-  for (long it = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
-       it += static_cast<long>(gridDim.x) * blockDim.x) {
-    const long t = it / per_row;
-    const int j = static_cast<int>(it % per_row);
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < topk; ++k) {
-      const long r = t * topk + k;
-      const int p = __ldg(pos + r);
-      if (p < 0) continue;
-      const float wk = w ? __ldg(w + r) : 1.f;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(D + static_cast<long>(p) * N) + j);
-      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+  for (long t = blockIdx.x; t < T; t += gridDim.x) {
+    int p[kCap];
+    float wk[kCap];
+#pragma unroll
+    for (int k = 0; k < kCap; ++k) {
+      p[k] = k < topk ? __ldg(pos + t * topk + k) : -1;
+      wk[k] = k < topk && w ? __ldg(w + t * topk + k) : 1.f;
+    }
+    for (int j = threadIdx.x; j < per_row; j += blockDim.x) {
+      uint4 v[kCap];
+#pragma unroll
+      for (int k = 0; k < kCap; ++k)
+        v[k] = p[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(D + static_cast<long>(p[k]) * N) + j)
+                         : make_uint4(0u, 0u, 0u, 0u);
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < kCap; ++k) {
+        if (p[k] < 0) continue;
+        const uint32_t wd[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] = fmaf(wk[k], __uint_as_float(wd[i] << 16), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(wk[k], __uint_as_float(wd[i] & 0xFFFF0000u), acc[2 * i + 1]);
+        }
+      }
+      uint4 o;
+      uint32_t* ow = &o.x;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        acc[2 * i] = fmaf(wk, __uint_as_float(wd[i] << 16), acc[2 * i]);
-        acc[2 * i + 1] = fmaf(wk, __uint_as_float(wd[i] & 0xFFFF0000u), acc[2 * i + 1]);
+        uint32_t packed;
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(packed) : "f"(acc[2 * i + 1]), "f"(acc[2 * i]));
+        ow[i] = packed;
       }
+      reinterpret_cast<uint4*>(out + t * N)[j] = o;
     }
-    uint4 o;
-    uint32_t* ow = &o.x;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t packed;
-      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(packed) : "f"(acc[2 * i + 1]), "f"(acc[2 * i]));
-      ow[i] = packed;
-    }
-    reinterpret_cast<uint4*>(out + t * N)[j] = o;
   }
 }
 
@@ -303,16 +314,22 @@ extern "C" int fp8g_moe_dispatch(const void* x, int x_dtype, int T, int K, const
 
 extern "C" int fp8g_moe_combine(const uint16_t* D, int N, const int32_t* pos, const float* w, int T, int topk,
                                 uint16_t* out, cudaStream_t stream) {
-  if (T < 0 || topk < 1 || N < 0) return FP8G_ERR_INVALID_ARG;
+  if (T < 0 || topk < 1 || topk > kMaxTopk || N < 0) return FP8G_ERR_INVALID_ARG;
   if (N % 8 != 0) return FP8G_ERR_MISALIGNED;
   if (T == 0 || N == 0) return FP8G_OK;
   if (!D || !pos || !out) return FP8G_ERR_INVALID_ARG;
   if (!aligned(D, 16) || !aligned(out, 16) || !aligned(pos, 4) || (w && !aligned(w, 4))) return FP8G_ERR_MISALIGNED;
   const int sms = sm_count();
   if (sms <= 0) return FP8G_ERR_CUDA;
-  const long items = static_cast<long>(T) * (N / 8);
-  const long blocks = std::min<long>((items + 255) / 256, 8L * sms);
-  moe_combine_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(D, N, pos, w, T, topk, out);
+  // a CTA per token: 256 threads, or fewer for narrow rows
+  const int threads = std::min(256, std::max(32, (N / 8 + 31) / 32 * 32));
+  const unsigned blocks = static_cast<unsigned>(std::min<long>(T, 16L * sms));
+  if (topk <= 4)
+    moe_combine_kernel<4><<<blocks, threads, 0, stream>>>(D, N, pos, w, T, topk, out);
+  else if (topk <= 8)
+    moe_combine_kernel<8><<<blocks, threads, 0, stream>>>(D, N, pos, w, T, topk, out);
+  else
+    moe_combine_kernel<kMaxTopk><<<blocks, threads, 0, stream>>>(D, N, pos, w, T, topk, out);
   if (cudaGetLastError() != cudaSuccess) return FP8G_ERR_CUDA;
   return FP8G_OK;
 }

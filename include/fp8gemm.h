@@ -272,8 +272,10 @@ int fp8g_moe_dispatch(const void *x, int x_dtype, int T, int K,
  * D[pos[t*topk + k]][n], accumulated in FP32 in slot order with one fused
  * multiply-add per slot (acc starts at 0; slots with pos < 0 are skipped;
  * w == NULL means weights of 1).  D [*][N] and out [T][N] are bf16 patterns,
- * N % 8 == 0, both 16-byte aligned.  With topk == 1 and w == NULL it returns
- * the GEMM's rows to token order.
+ * N % 8 == 0, both 16-byte aligned; 1 <= topk <= 16 (as for the dispatch).
+ * With topk == 1 and w == NULL it returns the GEMM's rows to token order.
+ * Errors: FP8G_ERR_INVALID_ARG (bad size or topk, null pointer),
+ * FP8G_ERR_MISALIGNED, FP8G_ERR_CUDA.
  */
 int fp8g_moe_combine(const uint16_t *D, int N, const int32_t *pos, const float *w,
                      int T, int topk, uint16_t *out, cudaStream_t stream);

@@ -175,3 +175,13 @@ def test_bf16_host_validation(lib):
     assert f(A + 8, B, D, 64, 256, 128, S) == 2     # A not 16-byte aligned
     assert f(None, B, D, 64, 256, 128, S) == 1      # null A
     assert f(None, None, None, 0, 256, 128, S) == 0  # M == 0: no-op
+
+
+def test_moe_combine_host_validation(lib):
+    f = lib.fp8g_moe_combine
+    f.argtypes = [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]
+    assert f(D, 64, A, None, 8, 17, D, S) == 1      # topk above 16
+    assert f(D, 64, A, None, 8, 0, D, S) == 1       # topk below 1
+    assert f(D, 60, A, None, 8, 4, D, S) == 2       # N % 8 != 0
+    assert f(None, 64, A, None, 8, 4, D, S) == 1    # null D
+    assert f(None, 64, None, None, 0, 4, None, S) == 0  # T == 0: no-op

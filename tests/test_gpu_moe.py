@@ -95,7 +95,7 @@ def test_dispatch_flags_bad_expert_ids(g):
     assert np.array_equal(p, epos) and np.array_equal(host(mi), emi)
 
 
-@pytest.mark.parametrize("T,topk,N", [(200, 1, 64), (333, 4, 520), (50, 8, 4096)])
+@pytest.mark.parametrize("T,topk,N", [(200, 1, 64), (333, 4, 520), (50, 8, 4096), (77, 12, 264)])
 def test_combine_matches_oracle_bit_for_bit(g, T, topk, N):
     rng = np.random.default_rng(T + N)
     G = max(6, topk)
