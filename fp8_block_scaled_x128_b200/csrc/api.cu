@@ -419,11 +419,11 @@ int launch(const Problem& P, int v, DeviceInfo* dev, cudaStream_t stream) {
     return FP8G_ERR_CUDA;
   }
   if (V.split == kGlobalSplitPartials) {
-    // the sum of the partials, one thread per 4 output elements
+    // the sum of the partials, one thread per output element
     cudaLaunchConfig_t rc_cfg = {};
     cudaLaunchAttribute rc_attr[1];
-    const long groups = static_cast<long>(p.num_tiles) * V.bnc * 32;
-    rc_cfg.gridDim = dim3(static_cast<unsigned>(std::min<long>((groups + 255) / 256, 4L * dev->sms)), 1, 1);
+    const long outputs = static_cast<long>(p.num_tiles) * V.bnc * 128;
+    rc_cfg.gridDim = dim3(static_cast<unsigned>(std::min<long>((outputs + 255) / 256, 4L * dev->sms)), 1, 1);
     rc_cfg.blockDim = dim3(256, 1, 1);
     rc_cfg.stream = stream;
     rc_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -806,33 +806,23 @@ template <int BNC>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const Params p) {
   grid_dependency_wait();
   if (threadIdx.x == 0) grid_launch_dependents();
-  // a thread sums 4 consecutive rows r of B (one 16-byte load per rank) and
-  // stores 4 consecutive columns n of D; N % 8 == 0, so a group is never cut
-  const long total = static_cast<long>(p.num_tiles) * BNC * 32;
+  const long total = static_cast<long>(p.num_tiles) * BNC * 128;
   const long stride = static_cast<long>(gridDim.x) * blockDim.x;
   for (long e = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += stride) {
-    const int tile = static_cast<int>(e / (BNC * 32));
-    const int c = static_cast<int>((e / 32) % BNC);
-    const int r0 = static_cast<int>(e % 32) * 4;
+    const int tile = static_cast<int>(e / (BNC * 128));
+    const int c = static_cast<int>((e / 128) % BNC);
+    const int r = static_cast<int>(e % 128);
     const int m = (tile / p.n_tiles) * BNC + c;
-    const int n0 = (tile % p.n_tiles) * 128 + r0;
-    if (m >= p.M || n0 >= p.N) continue;
-    const float4* src = reinterpret_cast<const float4*>(p.ws + static_cast<long>(tile) * p.gsplit * (BNC * 128) +
-                                                        c * 128 + r0);
-    float4 v[kMaxGSplit];
+    const int n = (tile % p.n_tiles) * 128 + r;
+    if (m >= p.M || n >= p.N) continue;
+    const float* src = p.ws + static_cast<long>(tile) * p.gsplit * (BNC * 128) + c * 128 + r;
+    float v[kMaxGSplit];
 #pragma unroll
-    for (int i = 0; i < kMaxGSplit; ++i)
-      v[i] = i < p.gsplit ? __ldcg(src + static_cast<long>(i) * (BNC * 32)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < kMaxGSplit; ++i) v[i] = i < p.gsplit ? __ldcg(src + static_cast<long>(i) * (BNC * 128)) : 0.f;
+    float sum = 0.f;
 #pragma unroll
-    for (int i = 0; i < kMaxGSplit; ++i) {  // rank order, as the single-element sum
-      sum.x += v[i].x;
-      sum.y += v[i].y;
-      sum.z += v[i].z;
-      sum.w += v[i].w;
-    }
-    *reinterpret_cast<uint2*>(p.D + static_cast<long>(m) * p.N + n0) =
-        make_uint2(pack_bf16x2(sum.x, sum.y), pack_bf16x2(sum.z, sum.w));
+    for (int i = 0; i < kMaxGSplit; ++i) sum += v[i];
+    p.D[static_cast<long>(m) * p.N + n] = static_cast<uint16_t>(pack_bf16x2(sum, 0.f) & 0xFFFFu);
   }
 }
 
